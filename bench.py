@@ -1,0 +1,391 @@
+#!/usr/bin/env python
+"""Benchmark: MoE-layer tokens/s for single-token decode of the 2-bit MoE FFN layer.
+
+Workload (one step): DECODE_BURST single-token decode passes (B = 1) through
+the decode layer -- d=4096, 256 routed experts (IQ2X gate/up, Q2K down),
+f=2048, top-8, bf16 shared expert f=2048 -- each pass = route + gate/up +
+down/combine.  Successive passes rotate over LAYERS resident layers, so the
+weights read between two uses of a layer (~330 MB) exceed the 126 MB L2: no
+flush is needed and none of a pass's weights is served from L2 by the previous
+pass.  The timed region replays a CUDA graph of one step K times.
+
+Also reported: the dominant kernel's roofline (the gate/up GEMV, HBM-bound),
+an end-to-end number through the public Python API with host<->device copies,
+the CPU oracle as baseline, and a prefill measurement (T=4096, grouped GEMM).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Multi-GPU: data-parallel replicas (each rank decodes its own token stream);
+no collective on the data path.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from bit_quantized_moe_02_b200 import synth  # noqa: E402
+
+DECODE_BURST = 256
+LAYERS = 4
+METRIC = "MoE-layer decode tokens/s (B=1)"
+UNIT = "tokens/s"
+
+
+def workload_config(wl, extra=None):
+    s = wl.shape
+    c = {"workload": "decode d=%d E=%d f=%d k=%d shared_f=%d B=1, IQ2X gate/up + Q2K down, bf16 shared"
+                     % (s.d, s.E, s.f, s.k, s.f_shared),
+         "tokens_per_step": DECODE_BURST, "layers_rotated": LAYERS,
+         "l2": "inputs larger than L2: %d layers rotated, %.0f MB of weights read per pass" % (
+             LAYERS, layer_bytes(wl) / 1e6)}
+    if extra:
+        c.update(extra)
+    return c
+
+
+def layer_bytes(wl):
+    """Algorithmic bytes of one B=1 decode pass: k experts' packed blocks, shared bf16 weights, router, x, out."""
+    s = wl.shape
+    routed = s.k * (2 * s.f * (s.d // 256) * 66 + s.d * (s.f // 256) * 84)
+    return routed + s.shared_bytes + s.router_bytes + s.d * 2 + s.d * 4
+
+
+def gateup_bytes(wl):
+    s = wl.shape
+    return s.k * 2 * s.f * (s.d // 256) * 66 + 2 * s.f_shared * s.d * 2 + s.d * 2
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return p["hbm_gbs"], p["bf16_tflops"], p.get("bf16_tflops_sustained"), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 50 ms while running."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.Q,
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out = ""
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in self.lines:
+            f = [v.strip() for v in l.split(",")]
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except (ValueError, IndexError):
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(args):
+    import torch
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600), device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v, ws):
+    if ws == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------------------------------------
+# CPU oracle legs
+
+
+def oracle_tokens_per_s(wl, n_tokens, nthreads, seed_stream=7):
+    """Time the oracle (as it stands) on n_tokens decode tokens of layer 0, nthreads host threads."""
+    import oracle
+    L = synth.make_layer(wl, layer=0)
+    x = synth.activations(wl, n_tokens, stream=seed_stream)
+    ids, _, _, _ = oracle.route(x, L.wr, L.bias, wl.shape.k)
+    for e in np.unique(ids):  # generate the touched experts before the clock starts
+        for w in ("gate", "up", "down"):
+            L.expert(w, int(e))
+    t0 = time.perf_counter()
+    oracle.layer_forward(L.shape, x, L.wr, L.bias, L.grid, L.expert, (L.sh_gate, L.sh_up, L.sh_down),
+                         nthreads=nthreads)
+    dt = time.perf_counter() - t0
+    return n_tokens / dt, dt
+
+
+def run_reference(args, ws, rank):
+    wl = synth.WORKLOADS["decode"]
+    if rank != 0:
+        return
+    cores = os.cpu_count() or 1
+    if args.warmup:
+        oracle_tokens_per_s(wl, min(args.warmup, cores), min(args.warmup, cores), seed_stream=8)
+    tps, dt = oracle_tokens_per_s(wl, args.steps, cores)
+    cb = {"value": tps, "unit": UNIT, "cores": min(cores, args.steps), "kind": "oracle",
+          "sample": "%d decode tokens (one per step), plain C oracle, fp32 dequant + fp64 contraction" % args.steps}
+    line = {"impl": "reference", "metric": METRIC, "value": tps, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(wl, {"tokens_per_step": 1}), "cpu_baseline": cb,
+            "e2e": {"value": tps, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------------------------------------
+# our arm
+
+
+def run_ours(args, ws, rank, local):
+    import torch
+    from bit_quantized_moe_02_b200 import ds4moe
+
+    torch.manual_seed(0)
+    wl = synth.WORKLOADS["decode"]
+    s = wl.shape
+    t_setup = time.perf_counter()
+    layers = [ds4moe.DeviceLayer(synth.make_layer(wl, layer=l + 16 * rank), max_tokens=1) for l in range(LAYERS)]
+    xs = [torch.from_numpy(synth.activations(wl, DECODE_BURST, layer=rank, stream=i)).cuda().view(torch.bfloat16)
+          for i in range(1)][0]
+    outs = torch.empty((DECODE_BURST, s.d), dtype=torch.float32, device="cuda")
+    ids_buf = torch.empty((DECODE_BURST, s.k), dtype=torch.int32, device="cuda")
+    w_buf = torch.empty((DECODE_BURST, s.k), dtype=torch.float32, device="cuda")
+    torch.cuda.synchronize()
+    setup_s = time.perf_counter() - t_setup
+
+    def one_pass(i):
+        Lr = layers[i % LAYERS]
+        ds4moe.route(xs[i:i + 1], Lr.wr, Lr.bias, s.k, ws=Lr.route_ws, ids=ids_buf[i:i + 1], weights=w_buf[i:i + 1])
+        ds4moe.expert_ffn_decode(Lr.ex, xs[i:i + 1], ids_buf[i:i + 1], w_buf[i:i + 1], Lr.ws, out=outs[i:i + 1])
+
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        for i in range(DECODE_BURST):  # eager warm-up of every launch
+            one_pass(i)
+        stream.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            for i in range(DECODE_BURST):
+                one_pass(i)
+        for _ in range(args.warmup):
+            graph.replay()
+        stream.synchronize()
+        assert ds4moe.last_device_error() == 0
+
+        # ---- timed region: exactly K steps (graph replays) ----
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(ws)
+        torch.cuda.synchronize()
+        with ClockSampler(local) as clk:
+            e0.record(stream)
+            for _ in range(args.steps):
+                graph.replay()
+            e1.record(stream)
+            torch.cuda.synchronize()
+        barrier(ws)
+        t_ms = e0.elapsed_time(e1)
+    t_max = max_over_ranks(t_ms, ws)
+    tokens = DECODE_BURST * args.steps * ws
+    value = tokens / (t_max / 1e3)
+
+    # ---- dominant kernel: gate/up GEMV, timed with events around each launch inside a graph ----
+    hbm, tf, tf_sus, peak_kind = peaks()
+    with torch.cuda.stream(stream):
+        ev = [(torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True),
+               torch.cuda.Event(enable_timing=True, external=True)) for _ in range(DECODE_BURST)]
+        g2 = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g2, stream=stream):
+            for i in range(DECODE_BURST):
+                Lr = layers[i % LAYERS]
+                ds4moe.route(xs[i:i + 1], Lr.wr, Lr.bias, s.k, ws=Lr.route_ws, ids=ids_buf[i:i + 1],
+                             weights=w_buf[i:i + 1])
+                ev[i][0].record(stream)
+                ds4moe.decode_gateup(Lr.ex, xs[i:i + 1], ids_buf[i:i + 1], Lr.ws)
+                ev[i][1].record(stream)
+                ds4moe.decode_down(Lr.ex, ids_buf[i:i + 1], w_buf[i:i + 1], Lr.ws, outs[i:i + 1])
+                ev[i][2].record(stream)
+        g2.replay()
+        g2.replay()
+        stream.synchronize()
+    gu_ms = float(np.mean([a.elapsed_time(b) for a, b, _ in ev]))
+    dn_ms = float(np.mean([b.elapsed_time(c) for _, b, c in ev]))
+    gu_bytes = gateup_bytes(wl)
+    achieved = gu_bytes / (gu_ms / 1e3) / 1e9
+    traffic = None
+    prof = os.path.join(ROOT, "profiles", "decode_gateup_traffic.json")
+    if os.path.exists(prof):
+        try:
+            traffic = json.load(open(prof)).get("bytes_per_launch")
+        except Exception:
+            traffic = None
+
+    # ---- end to end through the public API: pinned H2D of x, forward, D2H of the output, every step ----
+    n_e2e = min(DECODE_BURST, 256)
+    x_host = torch.from_numpy(synth.activations(wl, n_e2e, layer=rank, stream=5)).pin_memory()
+    out_host = torch.empty((1, s.d), dtype=torch.float32).pin_memory()
+    x_dev = torch.empty((1, s.d), dtype=torch.int16, device="cuda")
+    with torch.cuda.stream(stream):
+        for i in range(8):
+            layers[i % LAYERS].forward(x_dev.view(torch.bfloat16))
+        stream.synchronize()
+        barrier(ws)
+        t0 = time.perf_counter()
+        for i in range(n_e2e):
+            x_dev.copy_(x_host[i:i + 1], non_blocking=True)
+            o = layers[i % LAYERS].forward(x_dev.view(torch.bfloat16))
+            out_host.copy_(o, non_blocking=True)
+            stream.synchronize()
+        e2e_s = time.perf_counter() - t0
+    e2e_s = max_over_ranks(e2e_s, ws)
+    e2e_value = n_e2e * ws / e2e_s
+
+    # ---- prefill: T=4096 grouped path (one layer, eager) ----
+    prefill = None
+    if not args.no_prefill:
+        prefill = run_prefill(args, ds4moe, torch, stream, tf, tf_sus, peak_kind)
+
+    if rank != 0:
+        return
+    cpu = None
+    if ws == 1 and not args.no_cpu:
+        cores = os.cpu_count() or 1
+        tps, dt = oracle_tokens_per_s(wl, cores, cores)
+        cpu = {"value": tps, "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": "%d decode tokens of layer 0 (one per host thread), %.1f s" % (cores, dt)}
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": t_max / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f16 products / f32 accumulation (2-bit weights)", "data": "synthetic (seeded numpy; random-init weights)",
+        "config": workload_config(wl, {"parallelism": "replicas x%d" % ws if ws > 1 else "1 GPU"}),
+        "gpu_launches": 4 * DECODE_BURST * args.steps,
+        "layer_bytes_per_token": layer_bytes(wl),
+        "achieved_layer_GBps": layer_bytes(wl) * DECODE_BURST * args.steps / (t_ms / 1e3) / 1e9,
+        "roofline": {"bound": "hbm", "kernel": "decode_gateup_iq2x_kernel<16>", "achieved": achieved,
+                     "peak": hbm, "unit": "GB/s", "frac": achieved / hbm, "traffic": traffic,
+                     "peak_kind": peak_kind + " (burst copy)", "algorithmic_bytes_per_launch": gu_bytes,
+                     "avg_launch_ms": gu_ms, "down_kernel_avg_ms": dn_ms,
+                     "down_kernel_GBps": (layer_bytes(wl) - gu_bytes - s.router_bytes) / (dn_ms / 1e3) / 1e9},
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": s.d * 2, "d2h_bytes_per_step": s.d * 4,
+                "note": "one token per step through DeviceLayer.forward (route + decode), eager, sync per token"},
+        "clocks": clk.summary(),
+        "prefill": prefill,
+        "setup_s": setup_s,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_prefill(args, ds4moe, torch, stream, tf, tf_sus, peak_kind):
+    wl = synth.WORKLOADS["prefill"]
+    s = wl.shape
+    T = wl.tokens[0]
+    D = ds4moe.DeviceLayer(synth.make_layer(wl), max_tokens=T)
+    x = torch.from_numpy(synth.activations(wl, T)).cuda().view(torch.bfloat16)
+    y_perm = torch.empty((T * s.k, s.d), dtype=torch.float32, device="cuda")
+    inv = torch.empty(T * s.k, dtype=torch.int32, device="cuda")
+    ys = torch.empty((T, s.d), dtype=torch.float32, device="cuda")
+    out = torch.empty((T, s.d), dtype=torch.float32, device="cuda")
+    with torch.cuda.stream(stream):
+        def step():
+            ids, w = D.route(x)
+            ds4moe.expert_ffn_grouped(D.ex, x, ids, w, D.ws, y_perm, inv, ys)
+            ds4moe.combine(y_perm, inv, ys, T, s.d, s.k, out=out)
+        for _ in range(3):
+            step()
+        stream.synchronize()
+        n = 10
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n):
+            step()
+        e1.record(stream)
+        stream.synchronize()
+    ms = e0.elapsed_time(e1) / n
+    flops = 2 * 3 * s.d * s.f * T * s.k + 2 * 3 * s.d * s.f_shared * T + 2 * T * s.E * s.d
+    del D
+    return {"workload": "prefill T=%d, same layer, router bias N(0,1)" % T, "tokens_per_s": T / (ms / 1e3),
+            "ms_per_step": ms, "tflops": flops / (ms / 1e3) / 1e12,
+            "frac_of_bf16_peak": flops / (ms / 1e3) / 1e12 / tf, "peak_tflops": tf, "peak_kind": peak_kind}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        ws, rank = int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0"))
+        run_reference(args, ws, rank)
+        return
+    ws, rank, local = dist_setup(args)
+    try:
+        run_ours(args, ws, rank, local)
+    finally:
+        if ws > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,420 @@
+// Single-token decode: split-K GEMV over the selected experts' packed blocks.
+//
+// Kernel 1 (gate/up): every warp streams whole rows of an expert's gate and
+// up matrices (IQ2X, ~2.06 bits/weight) with coalesced 128-bit loads; each
+// lane owns a fixed slice of the contraction dimension whose activations stay
+// in registers as fp16 pairs.  8-vectors are dequantized in registers from a
+// shared-memory codebook table (lane-interleaved, conflict-free 128-bit
+// reads), signs are applied by XOR on the fp16 sign bits, products are
+// accumulated with packed fp16 FMAs inside one 32-weight group and in fp32
+// across groups; a warp-shuffle reduction finishes the row and the lane-0
+// epilogue applies SwiGLU.  The shared expert's gate/up rows (bf16) are split
+// into K-chunks and handled by the same warps, so the bandwidth-heavy bf16
+// stream and the ALU-heavy 2-bit stream overlap on every SM.
+//
+// Kernel 2 (down + combine): every CTA owns a range of output rows and loops
+// over the k routed experts (Q2K down rows) and the shared expert (bf16),
+// accumulating w_j * y_j + y_s in a fixed order (deterministic, no atomics).
+//
+// The method (only routed experts quantized; IQ2_XXS-style up/gate, Q2_K-style
+// down; shared expert unquantized) is the ds4 news summary's "model weights"
+// section; the kernel design is this library's own.
+#pragma once
+#include "common.cuh"
+
+namespace ds4 {
+
+struct ExpertsDev {
+    int d, f, E, fs;
+    int fmt_gate, fmt_down;
+    const uint8_t *gate, *up, *down;
+    uint64_t gate_stride, up_stride, down_stride;
+    const uint8_t *codebook;
+    const __nv_bfloat16 *sh_gate, *sh_up, *sh_down;
+    Planes pg;  // planes of one gate/up matrix [f x d]
+    Planes pd;  // planes of one down matrix [d x f]
+};
+
+constexpr int GU_THREADS = 384;
+constexpr int GU_TABLE_BYTES = 256 * 8 * 16;  // 8 lane-slots x 256 entries x 8 fp16
+
+// dynamic shared memory of the gate/up kernel: codebook table + fp32 copy of x
+__host__ __device__ constexpr int gu_smem_bytes(int d) { return GU_TABLE_BYTES + d * 4; }
+constexpr int DN_THREADS = 512;
+
+// Codebook table in shared memory: entry e, slot s (= lane & 7) at (e*8 + s)*16.
+__device__ __forceinline__ void build_codebook_table(const uint8_t *__restrict__ codebook, uint8_t *tbl) {
+    for (int i = threadIdx.x; i < 256 * 8; i += blockDim.x) {
+        int e = i >> 3;
+        const uint8_t *cb = codebook + e * 8;
+        __half2 h[4];
+#pragma unroll
+        for (int p = 0; p < 4; p++) h[p] = __floats2half2_rn(float(cb[2 * p]), float(cb[2 * p + 1]));
+        *reinterpret_cast<uint4 *>(tbl + size_t(i) * 16) = *reinterpret_cast<uint4 *>(h);
+    }
+}
+
+// Per-lane slice of one IQ2X row: VPL consecutive 8-vectors.
+template <int VPL>
+struct IqLane {
+    static constexpr int NG = VPL >= 4 ? VPL / 4 : 1;  // 32-weight groups touched
+    static constexpr int NW_IDX = (VPL + 3) / 4;       // u32 words of codebook indices
+    uint32_t idx[NW_IDX];
+    uint32_t sgn[NG];
+    uint32_t scl;
+    uint32_t dbits;
+};
+
+template <int VPL>
+__device__ __forceinline__ void iq_load(IqLane<VPL> &L, const uint8_t *__restrict__ mat, const Planes &P, int r,
+                                        int d, int lane) {
+    const int nsb = d / QK;
+    const uint8_t *ip = mat + P.off[0] + size_t(r) * (d / 8) + lane * VPL;
+    if constexpr (VPL == 16) {
+        uint4 v = ldg_nc_v4(ip);
+        L.idx[0] = v.x; L.idx[1] = v.y; L.idx[2] = v.z; L.idx[3] = v.w;
+    } else if constexpr (VPL == 8) {
+        uint2 v = *reinterpret_cast<const uint2 *>(ip);
+        L.idx[0] = v.x; L.idx[1] = v.y;
+    } else if constexpr (VPL == 4) {
+        L.idx[0] = ldg_nc_u32(ip);
+    } else if constexpr (VPL == 2) {
+        L.idx[0] = *reinterpret_cast<const uint16_t *>(ip);
+    } else {
+        L.idx[0] = *ip;
+    }
+    const uint8_t *sp = mat + P.off[1] + (size_t(r) * (d / 32) + (lane * VPL) / 4) * 4;
+    if constexpr (IqLane<VPL>::NG == 4) {
+        uint4 v = ldg_nc_v4(sp);
+        L.sgn[0] = v.x; L.sgn[1] = v.y; L.sgn[2] = v.z; L.sgn[3] = v.w;
+    } else if constexpr (IqLane<VPL>::NG == 2) {
+        uint2 v = *reinterpret_cast<const uint2 *>(sp);
+        L.sgn[0] = v.x; L.sgn[1] = v.y;
+    } else {
+        L.sgn[0] = ldg_nc_u32(sp);
+    }
+    const int sbi = (lane * VPL) / 32;
+    L.scl = ldg_nc_u32(mat + P.off[2] + (size_t(r) * nsb + sbi) * 4);
+    L.dbits = *reinterpret_cast<const uint16_t *>(mat + P.off[3] + (size_t(r) * nsb + sbi) * 2);
+}
+
+// Dot product of the lane's slice with its activations (scaled fp16 pairs).
+template <int VPL>
+__device__ __forceinline__ float iq_dot(const IqLane<VPL> &L, const uint32_t (&xh)[VPL][4], const uint8_t *tbl_lane,
+                                        int lane) {
+    constexpr uint32_t M = 0x80008000u;
+    constexpr int NV = VPL < 4 ? VPL : 4;
+    const int g0 = ((lane * VPL) / 4) % 8;
+    const int j0 = VPL < 4 ? (lane * VPL) % 4 : 0;
+    const float dv = half_bits_to_float(uint16_t(L.dbits));
+    float acc = 0.f;
+#pragma unroll
+    for (int gi = 0; gi < IqLane<VPL>::NG; gi++) {
+        const uint32_t W = L.sgn[gi];
+        const float s = float((L.scl >> (4 * (g0 + gi))) & 15u);
+        const float Dg = (dv * (0.5f + s)) * 0.25f;
+        __half2 a0 = __float2half2_rn(0.f), a1 = __float2half2_rn(0.f);
+#pragma unroll
+        for (int jj = 0; jj < NV; jj++) {
+            const int v = gi * 4 + jj;
+            const int j = j0 + jj;
+            const uint32_t ib = (L.idx[v / 4] >> (8 * (v % 4))) & 0xFFu;
+            const uint4 cb = *reinterpret_cast<const uint4 *>(tbl_lane + ib * 128);
+            const uint32_t Wj = W << (4 * j);
+            const uint32_t c0 = cb.x ^ (Wj & M);
+            const uint32_t c1 = cb.y ^ ((Wj << 1) & M);
+            const uint32_t c2 = cb.z ^ ((Wj << 2) & M);
+            const uint32_t c3 = cb.w ^ ((Wj << 3) & M);
+            a0 = __hfma2(u32_as_half2(c0), u32_as_half2(xh[v][0]), a0);
+            a1 = __hfma2(u32_as_half2(c1), u32_as_half2(xh[v][1]), a1);
+            a0 = __hfma2(u32_as_half2(c2), u32_as_half2(xh[v][2]), a0);
+            a1 = __hfma2(u32_as_half2(c3), u32_as_half2(xh[v][3]), a1);
+        }
+        const float2 f0 = __half22float2(a0), f1 = __half22float2(a1);
+        acc = fmaf(Dg, (f0.x + f0.y) + (f1.x + f1.y), acc);
+    }
+    return acc;
+}
+
+// Block-wide max of |x| over d bf16 values -> power-of-two exponent putting it in [32, 64).
+__device__ __forceinline__ int block_x_exponent(const __nv_bfloat16 *__restrict__ x, int d, float *red) {
+    float m = 0.f;
+    for (int i = threadIdx.x; i < d; i += blockDim.x) m = fmaxf(m, fabsf(__bfloat162float(x[i])));
+    m = warp_max(m);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    if (lane == 0) red[warp] = m;
+    __syncthreads();
+    float v = lane < nw ? red[lane] : 0.f;
+    v = warp_max(v);
+    __syncthreads();
+    return pow2_exponent_for(v, 6);
+}
+
+// h_out[j*f + r] = silu(g) * u for routed slot j; sh_part[(2c+{0,1})*fs + r] = chunk-c partial g/u of the shared expert.
+template <int VPL>
+__global__ void __launch_bounds__(GU_THREADS, 1)
+    decode_gateup_iq2x_kernel(ExpertsDev ex, const __nv_bfloat16 *__restrict__ x, const int32_t *__restrict__ ids,
+                              int k, float *__restrict__ h_out, float *__restrict__ sh_part) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    __shared__ float red[32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    constexpr int NWARP = GU_THREADS / 32;
+    const int d = ex.d;
+
+    build_codebook_table(ex.codebook, smem);
+    const int xe = block_x_exponent(x, d, red);  // includes __syncthreads (table visible)
+    const float xs = ldexpf(1.f, xe), inv_xs = ldexpf(1.f, -xe);
+
+    uint32_t xh[VPL][4];
+#pragma unroll
+    for (int v = 0; v < VPL; v++) {
+        uint4 raw = *reinterpret_cast<const uint4 *>(x + size_t(lane * VPL + v) * 8);
+        const uint32_t rw[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+        for (int i = 0; i < 4; i++) xh[v][i] = half2_as_u32(__floats2half2_rn(bf16_lo(rw[i]) * xs, bf16_hi(rw[i]) * xs));
+    }
+    const uint8_t *tbl_lane = smem + (lane & 7) * 16;
+
+    constexpr int NCV = VPL < 4 ? VPL : 4;  // 8-vectors per lane per shared-expert chunk
+    constexpr int NCH = VPL / NCV;          // chunks per shared row
+    constexpr int EL = 8 * NCV;             // elements per lane per chunk
+    constexpr int CS = 32 * EL;             // elements per chunk
+    // x for the shared expert: element c*CS + l*EL + 4i + q at float4 slot (c*EL/4 + i)*32 + l, component q
+    float4 *xsh = reinterpret_cast<float4 *>(smem + GU_TABLE_BYTES);
+    for (int q4 = threadIdx.x; q4 < d / 4; q4 += blockDim.x) {
+        const int el = q4 * 4, c = el / CS, l = (el % CS) / EL, i = (el % EL) / 4;
+        const uint2 raw = *reinterpret_cast<const uint2 *>(x + el);
+        xsh[(c * (EL / 4) + i) * 32 + l] = make_float4(bf16_lo(raw.x), bf16_hi(raw.x), bf16_lo(raw.y), bf16_hi(raw.y));
+    }
+    __syncthreads();
+    const int n_sh = ex.fs > 0 ? ex.fs * NCH : 0;
+    const int n_items = n_sh + k * ex.f;
+    const int nw_total = gridDim.x * NWARP;
+    bool waited = false;
+    for (int it = blockIdx.x * NWARP + warp; it < n_items; it += nw_total) {
+        if (it < n_sh) {
+            // lane handles elements [c*CS + lane*EL, +EL) of the row; x comes from shared memory
+            const int r = it / NCH, c = it % NCH;
+            const size_t off = size_t(r) * d + size_t(c) * CS + size_t(lane) * EL;
+            uint4 gv[NCV], uv[NCV];
+#pragma unroll
+            for (int v = 0; v < NCV; v++) {
+                gv[v] = ldg_nc_v4(ex.sh_gate + off + 8 * v);
+                uv[v] = ldg_nc_v4(ex.sh_up + off + 8 * v);
+            }
+            float ag = 0.f, au = 0.f;
+#pragma unroll
+            for (int v = 0; v < NCV; v++) {
+                const float4 xa = xsh[(c * (EL / 4) + 2 * v) * 32 + lane];
+                const float4 xb = xsh[(c * (EL / 4) + 2 * v + 1) * 32 + lane];
+                const float xf[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+                const uint32_t gw[4] = {gv[v].x, gv[v].y, gv[v].z, gv[v].w};
+                const uint32_t uw[4] = {uv[v].x, uv[v].y, uv[v].z, uv[v].w};
+#pragma unroll
+                for (int i = 0; i < 4; i++) {
+                    ag = fmaf(bf16_lo(gw[i]), xf[2 * i], ag);
+                    ag = fmaf(bf16_hi(gw[i]), xf[2 * i + 1], ag);
+                    au = fmaf(bf16_lo(uw[i]), xf[2 * i], au);
+                    au = fmaf(bf16_hi(uw[i]), xf[2 * i + 1], au);
+                }
+            }
+            ag = warp_sum(ag);
+            au = warp_sum(au);
+            if (lane == 0) {
+                sh_part[size_t(2 * c) * ex.fs + r] = ag;
+                sh_part[size_t(2 * c + 1) * ex.fs + r] = au;
+            }
+        } else {
+            if (!waited) {
+                pdl_wait();
+                waited = true;
+            }
+            const int q = it - n_sh;
+            const int j = q / ex.f, r = q % ex.f;
+            const int e = ids[j];
+            if (e < 0 || e >= ex.E) {
+                if (lane == 0) set_device_error(DS4MOE_EDEVICE);
+                continue;
+            }
+            IqLane<VPL> Lg, Lu;
+            iq_load<VPL>(Lg, ex.gate + size_t(e) * ex.gate_stride, ex.pg, r, d, lane);
+            iq_load<VPL>(Lu, ex.up + size_t(e) * ex.up_stride, ex.pg, r, d, lane);
+            float ag = iq_dot<VPL>(Lg, xh, tbl_lane, lane);
+            float au = iq_dot<VPL>(Lu, xh, tbl_lane, lane);
+            ag = warp_sum(ag);
+            au = warp_sum(au);
+            if (lane == 0) {
+                const float g = ag * inv_xs, u = au * inv_xs;
+                h_out[size_t(j) * ex.f + r] = silu(g) * u;
+            }
+        }
+    }
+}
+
+// ---- down + combine -------------------------------------------------------
+
+struct DownSmem {
+    // offsets (bytes) inside dynamic shared memory
+    int hq, hsum, hsl, wsc, eid, total;
+};
+
+__host__ __device__ __forceinline__ DownSmem down_smem_layout(int k, int wpl, int fs) {
+    DownSmem s;
+    s.hq = 0;                                     // k * wpl * 2 * 32 uint4
+    s.hsum = s.hq + k * wpl * 2 * 32 * 16;         // k * wpl * 32 float
+    s.hsl = s.hsum + k * wpl * 32 * 4;             // fs floats (lane-interleaved float4s)
+    s.wsc = s.hsl + ((fs * 4 + 15) / 16) * 16;     // k floats
+    s.eid = s.wsc + ((k * 4 + 15) / 16) * 16;      // k ints
+    s.total = s.eid + ((k * 4 + 15) / 16) * 16;
+    return s;
+}
+
+// out[n] = sum_j w_j * (D_{e_j} h_j)[n] + (Ds hs)[n], hs = silu(sum_c gpart) * sum_c upart.
+template <int WPL>
+__global__ void __launch_bounds__(DN_THREADS, 1)
+    decode_down_q2k_kernel(ExpertsDev ex, const float *__restrict__ h, const float *__restrict__ sh_part, int nch,
+                           const int32_t *__restrict__ ids, const float *__restrict__ wts, int k,
+                           float *__restrict__ out) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    constexpr int NWARP = DN_THREADS / 32;
+    const int f = ex.f, fs = ex.fs, d = ex.d;
+    const int nwords = f / 16;
+    const int active = nwords < 32 ? nwords : 32;
+    const DownSmem L = down_smem_layout(k, WPL, fs);
+    uint4 *hq = reinterpret_cast<uint4 *>(smem + L.hq);
+    float *hsum = reinterpret_cast<float *>(smem + L.hsum);
+    float *hsl = reinterpret_cast<float *>(smem + L.hsl);
+    float *wsc = reinterpret_cast<float *>(smem + L.wsc);
+    int *eid = reinterpret_cast<int *>(smem + L.eid);
+
+    pdl_wait();
+    // stage routed h_j as scaled fp16 pairs (h[16s+p], h[16s+p+8]) in lane-interleaved order
+    for (int j = warp; j < k; j += NWARP) {
+        const float *hj = h + size_t(j) * f;
+        float mx = 0.f;
+        if (lane < active)
+            for (int i = 0; i < WPL; i++)
+                for (int e = 0; e < 16; e++) mx = fmaxf(mx, fabsf(hj[(lane * WPL + i) * 16 + e]));
+        mx = warp_max(mx);
+        const int he = pow2_exponent_for(mx, 6);
+        const float sc = ldexpf(1.f, he);
+        if (lane < active) {
+            for (int i = 0; i < WPL; i++) {
+                const float *src = hj + (lane * WPL + i) * 16;
+                __half2 pr[8];
+                float ssum = 0.f;
+#pragma unroll
+                for (int p = 0; p < 8; p++) {
+                    pr[p] = __floats2half2_rn(src[p] * sc, src[p + 8] * sc);
+                    const float2 back = __half22float2(pr[p]);
+                    ssum += back.x + back.y;
+                }
+                hq[((j * WPL + i) * 2 + 0) * 32 + lane] = *reinterpret_cast<uint4 *>(&pr[0]);
+                hq[((j * WPL + i) * 2 + 1) * 32 + lane] = *reinterpret_cast<uint4 *>(&pr[4]);
+                hsum[(j * WPL + i) * 32 + lane] = ssum;
+            }
+        }
+        if (lane == 0) {
+            wsc[j] = wts[j] * ldexpf(1.f, -he);
+            eid[j] = ids[j];
+        }
+    }
+    // shared expert: hs = silu(g) * u, element r at lane r/ESL, offset o = r%ESL -> float4 slot [o/4][lane]
+    const int esl = fs / 32;
+    for (int r = threadIdx.x; r < fs; r += blockDim.x) {
+        float g = 0.f, u = 0.f;
+        for (int c = 0; c < nch; c++) {
+            g += sh_part[size_t(2 * c) * fs + r];
+            u += sh_part[size_t(2 * c + 1) * fs + r];
+        }
+        const int ln = r / esl, o = r % esl;
+        hsl[((o / 4) * 32 + ln) * 4 + (o % 4)] = silu(g) * u;
+    }
+    __syncthreads();
+
+    const int rpc = (d + gridDim.x - 1) / gridDim.x;
+    const int n0 = blockIdx.x * rpc, n1 = min(d, n0 + rpc);
+    const int nsbf = f / QK;
+    const __half2 k1024 = __float2half2_rn(1024.f);
+    for (int n = n0 + warp; n < n1; n += NWARP) {
+        float acc = 0.f;
+        if (lane < active) {
+#pragma unroll 2
+            for (int j = 0; j < k; j++) {
+                const int e = eid[j];
+                if (e < 0 || e >= ex.E) {
+                    if (lane == 0) set_device_error(DS4MOE_EDEVICE);
+                    continue;
+                }
+                const uint8_t *base = ex.down + size_t(e) * ex.down_stride;
+                const uint8_t *qp = base + ex.pd.off[0] + size_t(n) * nsbf * 64 + lane * WPL * 4;
+                const uint8_t *sp = base + ex.pd.off[1] + size_t(n) * nsbf * 16 + lane * WPL;
+                const uint32_t dm =
+                    ldg_nc_u32(base + ex.pd.off[2] + (size_t(n) * nsbf + (lane * WPL) / 16) * 4);
+                uint32_t qw[WPL];
+                uint32_t scw[(WPL + 3) / 4];
+                if constexpr (WPL == 8) {
+                    uint4 a = ldg_nc_v4(qp), b = ldg_nc_v4(qp + 16);
+                    qw[0] = a.x; qw[1] = a.y; qw[2] = a.z; qw[3] = a.w;
+                    qw[4] = b.x; qw[5] = b.y; qw[6] = b.z; qw[7] = b.w;
+                    uint2 s2 = *reinterpret_cast<const uint2 *>(sp);
+                    scw[0] = s2.x; scw[1] = s2.y;
+                } else if constexpr (WPL == 4) {
+                    uint4 a = ldg_nc_v4(qp);
+                    qw[0] = a.x; qw[1] = a.y; qw[2] = a.z; qw[3] = a.w;
+                    scw[0] = ldg_nc_u32(sp);
+                } else if constexpr (WPL == 2) {
+                    uint2 a = *reinterpret_cast<const uint2 *>(qp);
+                    qw[0] = a.x; qw[1] = a.y;
+                    scw[0] = *reinterpret_cast<const uint16_t *>(sp);
+                } else {
+                    qw[0] = ldg_nc_u32(qp);
+                    scw[0] = *sp;
+                }
+                const float dd = half_bits_to_float(uint16_t(dm & 0xFFFF));
+                const float dmin = half_bits_to_float(uint16_t(dm >> 16));
+                float part = 0.f;
+#pragma unroll
+                for (int i = 0; i < WPL; i++) {
+                    const uint4 hA = hq[((j * WPL + i) * 2 + 0) * 32 + lane];
+                    const uint4 hB = hq[((j * WPL + i) * 2 + 1) * 32 + lane];
+                    const uint32_t hp[8] = {hA.x, hA.y, hA.z, hA.w, hB.x, hB.y, hB.z, hB.w};
+                    __half2 a = __float2half2_rn(0.f), b = __float2half2_rn(0.f);
+#pragma unroll
+                    for (int p = 0; p < 8; p++) {
+                        const uint32_t v = ((qw[i] >> (2 * p)) & 0x00030003u) | 0x64006400u;
+                        const __half2 q2 = __hsub2(u32_as_half2(v), k1024);
+                        if (p & 1) b = __hfma2(q2, u32_as_half2(hp[p]), b);
+                        else a = __hfma2(q2, u32_as_half2(hp[p]), a);
+                    }
+                    const float2 fa = __half22float2(a), fb = __half22float2(b);
+                    const uint32_t scb = (scw[i / 4] >> (8 * (i % 4))) & 0xFFu;
+                    const float sc = float(scb & 15u), mn = float(scb >> 4);
+                    part += (dd * sc) * ((fa.x + fa.y) + (fb.x + fb.y)) - (dmin * mn) * hsum[(j * WPL + i) * 32 + lane];
+                }
+                acc = fmaf(wsc[j], part, acc);
+            }
+        }
+        if (fs > 0) {
+            const __nv_bfloat16 *row = ex.sh_down + size_t(n) * fs + size_t(lane) * esl;
+            const float4 *h4 = reinterpret_cast<const float4 *>(hsl);
+            for (int i = 0; i < esl / 8; i++) {
+                const uint4 wv = ldg_nc_v4(row + 8 * i);
+                const float4 ha = h4[(2 * i) * 32 + lane], hb = h4[(2 * i + 1) * 32 + lane];
+                acc = fmaf(bf16_lo(wv.x), ha.x, acc);
+                acc = fmaf(bf16_hi(wv.x), ha.y, acc);
+                acc = fmaf(bf16_lo(wv.y), ha.z, acc);
+                acc = fmaf(bf16_hi(wv.y), ha.w, acc);
+                acc = fmaf(bf16_lo(wv.z), hb.x, acc);
+                acc = fmaf(bf16_hi(wv.z), hb.y, acc);
+                acc = fmaf(bf16_lo(wv.w), hb.z, acc);
+                acc = fmaf(bf16_hi(wv.w), hb.w, acc);
+            }
+        }
+        acc = warp_sum(acc);
+        if (lane == 0) out[n] = acc;
+    }
+}
+
+}  // namespace ds4

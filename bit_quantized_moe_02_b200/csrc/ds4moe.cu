@@ -1,0 +1,491 @@
+// ds4moe C ABI (include/ds4moe.h): argument checks, workspace carving and
+// kernel launches.  One translation unit: the kernels live in the headers
+// included below.
+#include <stdio.h>
+
+#include "common.cuh"
+#include "decode.cuh"
+#include "grouped_mma.cuh"
+#include "permute.cuh"
+#include "prepare.cuh"
+#include "route.cuh"
+
+using namespace ds4;
+
+namespace {
+
+#define DS4_CHECK_LAUNCH()                                          \
+    do {                                                            \
+        if (cudaGetLastError() != cudaSuccess) return DS4MOE_ECUDA; \
+    } while (0)
+
+inline cudaStream_t cs(ds4moe_stream s) { return reinterpret_cast<cudaStream_t>(s); }
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+inline bool aligned256(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 255) == 0; }
+inline uint64_t a256(uint64_t x) { return (x + 255) & ~uint64_t(255); }
+
+int num_sms() {
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (dev < 64 && cache[dev]) return cache[dev];
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    if (dev < 64) cache[dev] = n;
+    return n;
+}
+
+// Opt in to the dynamic shared memory a kernel needs (static + dynamic above 48 KB needs the attribute).
+template <typename Kern>
+bool set_smem(Kern k, int bytes) {
+    return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
+}
+
+// Launch with programmatic dependent launch enabled (the kernel calls pdl_wait before consuming
+// the previous kernel's results).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
+bool fmt_quant(int f) { return f == DS4MOE_FMT_IQ2X || f == DS4MOE_FMT_Q2K || f == DS4MOE_FMT_Q4K; }
+
+ds4moe_status check_experts(const ds4moe_experts *ex) {
+    if (!ex) return DS4MOE_EINVAL;
+    if (ex->d <= 0 || ex->f <= 0 || ex->E <= 0 || ex->d % QK || ex->f % QK || ex->f_shared < 0 ||
+        ex->f_shared % QK)
+        return DS4MOE_EINVAL;
+    if (!fmt_quant(ex->fmt_gate) || !fmt_quant(ex->fmt_down) || ex->fmt_up != ex->fmt_gate) return DS4MOE_EUNSUPPORTED;
+    if (ex->fmt_gate == DS4MOE_FMT_Q2K) return DS4MOE_EUNSUPPORTED;  // gate/up: IQ2X or Q4K
+    if (ex->fmt_down == DS4MOE_FMT_IQ2X) return DS4MOE_EUNSUPPORTED;  // down: Q2K or Q4K
+    if (!ex->gate || !ex->up || !ex->down) return DS4MOE_EINVAL;
+    if (!aligned256(ex->gate) || !aligned256(ex->up) || !aligned256(ex->down)) return DS4MOE_EINVAL;
+    const uint64_t gb = ds4moe_prepared_bytes(ds4moe_fmt(ex->fmt_gate), ex->f, ex->d);
+    const uint64_t db = ds4moe_prepared_bytes(ds4moe_fmt(ex->fmt_down), ex->d, ex->f);
+    if (ex->gate_stride < gb || ex->up_stride < gb || ex->down_stride < db) return DS4MOE_EINVAL;
+    if (ex->gate_stride % 256 || ex->up_stride % 256 || ex->down_stride % 256) return DS4MOE_EINVAL;
+    if (ex->fmt_gate == DS4MOE_FMT_IQ2X && (!ex->codebook || !aligned16(ex->codebook))) return DS4MOE_EINVAL;
+    if (ex->f_shared > 0) {
+        if (!ex->sh_gate || !ex->sh_up || !ex->sh_down) return DS4MOE_EINVAL;
+        if (!aligned16(ex->sh_gate) || !aligned16(ex->sh_up) || !aligned16(ex->sh_down)) return DS4MOE_EINVAL;
+    }
+    return DS4MOE_OK;
+}
+
+ExpertsDev to_dev(const ds4moe_experts *ex) {
+    ExpertsDev e;
+    e.d = ex->d; e.f = ex->f; e.E = ex->E; e.fs = ex->f_shared;
+    e.fmt_gate = ex->fmt_gate; e.fmt_down = ex->fmt_down;
+    e.gate = static_cast<const uint8_t *>(ex->gate);
+    e.up = static_cast<const uint8_t *>(ex->up);
+    e.down = static_cast<const uint8_t *>(ex->down);
+    e.gate_stride = ex->gate_stride; e.up_stride = ex->up_stride; e.down_stride = ex->down_stride;
+    e.codebook = ex->codebook;
+    e.sh_gate = static_cast<const __nv_bfloat16 *>(ex->sh_gate);
+    e.sh_up = static_cast<const __nv_bfloat16 *>(ex->sh_up);
+    e.sh_down = static_cast<const __nv_bfloat16 *>(ex->sh_down);
+    e.pg = plane_layout(ex->fmt_gate, uint64_t(ex->f) * (ex->d / QK));
+    e.pd = plane_layout(ex->fmt_down, uint64_t(ex->d) * (ex->f / QK));
+    return e;
+}
+
+// ---- workspace layouts -----------------------------------------------------------------------------
+
+bool decode_gemv_supported(const ds4moe_experts *ex, int k) {
+    const int vpl = ex->d / QK, wpl = ex->f / 512;
+    const bool vpl_ok = vpl == 1 || vpl == 2 || vpl == 4 || vpl == 8 || vpl == 16;
+    const bool wpl_ok = ex->f == 256 || wpl == 1 || wpl == 2 || wpl == 4 || wpl == 8;
+    return ex->fmt_gate == DS4MOE_FMT_IQ2X && ex->fmt_down == DS4MOE_FMT_Q2K && vpl_ok && wpl_ok && k <= 32;
+}
+
+struct DecodeWs {
+    uint64_t h, sh_part, total;
+    int nch;
+};
+DecodeWs decode_ws(const ds4moe_experts *ex, int k) {
+    DecodeWs w;
+    const int vpl = ex->d / QK;
+    const int ncv = vpl < 4 ? vpl : 4;
+    w.nch = vpl / ncv;
+    w.h = 0;
+    w.sh_part = a256(uint64_t(k) * ex->f * 4);
+    w.total = w.sh_part + a256(uint64_t(w.nch) * 2 * (ex->f_shared > 0 ? ex->f_shared : 1) * 4);
+    return w;
+}
+
+struct GroupedWs {
+    uint64_t x16, xinv, blk, counts, offsets, tile_e, tile_pos0, tile_cnt, meta, perm_tok, perm_w, h16, hs;
+    uint64_t y_perm, inv, y_shared;  // only used when decode B > 1 runs through the grouped path
+    uint64_t total_grouped, total_decode;
+    int nblk, max_tiles;
+};
+GroupedWs grouped_ws(const ds4moe_experts *ex, int T, int k) {
+    GroupedWs w;
+    const uint64_t N = uint64_t(T) * k;
+    w.nblk = int((N + PERM_BLOCK - 1) / PERM_BLOCK);
+    w.max_tiles = int(ex->E + (N + TILE_N - 1) / TILE_N);
+    uint64_t o = 0;
+    auto take = [&](uint64_t bytes) {
+        uint64_t r = o;
+        o += a256(bytes > 0 ? bytes : 1);
+        return r;
+    };
+    w.x16 = take(uint64_t(T) * ex->d * 2);
+    w.xinv = take(uint64_t(T) * 4);
+    w.blk = take(uint64_t(w.nblk > 0 ? w.nblk : 1) * ex->E * 4);
+    w.counts = take(uint64_t(ex->E) * 4);
+    w.offsets = take(uint64_t(ex->E) * 4);
+    w.tile_e = take(uint64_t(w.max_tiles) * 4);
+    w.tile_pos0 = take(uint64_t(w.max_tiles) * 4);
+    w.tile_cnt = take(uint64_t(w.max_tiles) * 4);
+    w.meta = take(16);
+    w.perm_tok = take(N * 4);
+    w.perm_w = take(N * 4);
+    w.h16 = take(N * ex->f * 2);
+    w.hs = take(uint64_t(T) * (ex->f_shared > 0 ? ex->f_shared : 1) * 2);
+    w.total_grouped = o;
+    w.y_perm = take(N * ex->d * 4);
+    w.inv = take(N * 4);
+    w.y_shared = take(uint64_t(T) * ex->d * 4);
+    w.total_decode = o;
+    return w;
+}
+
+// ---- grouped launch sequence --------------------------------------------------------------------------
+
+template <int AFMT, bool GATEUP>
+ds4moe_status launch_grouped(const GroupedArgs &ga, int row_tiles, int col_tiles, cudaStream_t st) {
+    auto kern = grouped_mma_kernel<AFMT, GATEUP>;
+    if (!set_smem(kern, GM_SMEM)) return DS4MOE_ECUDA;
+    if (row_tiles <= 0 || col_tiles <= 0) return DS4MOE_OK;
+    kern<<<dim3(row_tiles, col_tiles), GM_THREADS, GM_SMEM, st>>>(ga);
+    DS4_CHECK_LAUNCH();
+    return DS4MOE_OK;
+}
+
+ds4moe_status run_grouped(const ds4moe_experts *ex, const void *x, int T, const int32_t *ids, const float *weights,
+                          int k, float *y_perm, int32_t *inv_perm, float *y_shared, uint8_t *ws, cudaStream_t st) {
+    const GroupedWs W = grouped_ws(ex, T, k);
+    const ExpertsDev D = to_dev(ex);
+    const int N = T * k;
+    __half *x16 = reinterpret_cast<__half *>(ws + W.x16);
+    float *xinv = reinterpret_cast<float *>(ws + W.xinv);
+    int32_t *blk = reinterpret_cast<int32_t *>(ws + W.blk);
+    int32_t *counts = reinterpret_cast<int32_t *>(ws + W.counts);
+    int32_t *offsets = reinterpret_cast<int32_t *>(ws + W.offsets);
+    int32_t *tile_e = reinterpret_cast<int32_t *>(ws + W.tile_e);
+    int32_t *tile_pos0 = reinterpret_cast<int32_t *>(ws + W.tile_pos0);
+    int32_t *tile_cnt = reinterpret_cast<int32_t *>(ws + W.tile_cnt);
+    int32_t *meta = reinterpret_cast<int32_t *>(ws + W.meta);
+    int32_t *perm_tok = reinterpret_cast<int32_t *>(ws + W.perm_tok);
+    float *perm_w = reinterpret_cast<float *>(ws + W.perm_w);
+    __half *h16 = reinterpret_cast<__half *>(ws + W.h16);
+    __half *hs = reinterpret_cast<__half *>(ws + W.hs);
+    const __nv_bfloat16 *xb = static_cast<const __nv_bfloat16 *>(x);
+
+    prep_x_kernel<<<T, 256, 0, st>>>(xb, ex->d, x16, xinv);
+    DS4_CHECK_LAUNCH();
+    const size_t hist_smem = size_t(ex->E) * 4;
+    perm_count_kernel<<<W.nblk, PERM_BLOCK, hist_smem, st>>>(ids, N, ex->E, blk);
+    DS4_CHECK_LAUNCH();
+    perm_scan_kernel<<<1, 1024, 0, st>>>(blk, W.nblk, ex->E, counts, offsets, tile_e, tile_pos0, tile_cnt, meta);
+    DS4_CHECK_LAUNCH();
+    perm_scatter_kernel<<<W.nblk, PERM_BLOCK, hist_smem, st>>>(ids, weights, N, k, ex->E, blk, perm_tok, perm_w,
+                                                               inv_perm);
+    DS4_CHECK_LAUNCH();
+
+    // routed GEMM-1: gate/up -> h16
+    GroupedArgs g1 = {};
+    g1.a0 = D.gate; g1.a1 = D.up; g1.a_stride = D.gate_stride; g1.pa = D.pg;
+    g1.rows = ex->f; g1.K = ex->d; g1.codebook = ex->codebook;
+    g1.b_src = x16; g1.b_rowidx = perm_tok; g1.b_colscale = xinv;
+    g1.tile_e = tile_e; g1.tile_pos0 = tile_pos0; g1.tile_cnt = tile_cnt; g1.n_tiles = meta;
+    g1.out = h16; g1.ldo = ex->f;
+    ds4moe_status s;
+    if (ex->fmt_gate == DS4MOE_FMT_IQ2X) s = launch_grouped<DS4MOE_FMT_IQ2X, true>(g1, ex->f / 64, W.max_tiles, st);
+    else s = launch_grouped<DS4MOE_FMT_Q4K, true>(g1, ex->f / 64, W.max_tiles, st);
+    if (s != DS4MOE_OK) return s;
+
+    // routed GEMM-2: down -> y_perm (scaled by the routing weight)
+    GroupedArgs g2 = {};
+    g2.a0 = D.down; g2.a_stride = D.down_stride; g2.pa = D.pd; g2.rows = ex->d; g2.K = ex->f;
+    g2.b_src = h16; g2.b_rowidx = nullptr; g2.b_colscale = nullptr;
+    g2.tile_e = tile_e; g2.tile_pos0 = tile_pos0; g2.tile_cnt = tile_cnt; g2.n_tiles = meta;
+    g2.pos_weight = perm_w; g2.out = y_perm; g2.ldo = ex->d;
+    if (ex->fmt_down == DS4MOE_FMT_Q2K) s = launch_grouped<DS4MOE_FMT_Q2K, false>(g2, ex->d / GM_M, W.max_tiles, st);
+    else s = launch_grouped<DS4MOE_FMT_Q4K, false>(g2, ex->d / GM_M, W.max_tiles, st);
+    if (s != DS4MOE_OK) return s;
+
+    if (ex->f_shared > 0) {
+        const int ct = (T + GM_N - 1) / GM_N;
+        GroupedArgs s1 = {};
+        s1.a0 = static_cast<const uint8_t *>(ex->sh_gate); s1.a1 = static_cast<const uint8_t *>(ex->sh_up);
+        s1.a_stride = 0; s1.rows = ex->f_shared; s1.K = ex->d;
+        s1.b_src = x16; s1.b_colscale = xinv; s1.n_pos = T; s1.out = hs; s1.ldo = ex->f_shared;
+        s = launch_grouped<DS4MOE_FMT_BF16, true>(s1, ex->f_shared / 64, ct, st);
+        if (s != DS4MOE_OK) return s;
+        GroupedArgs s2 = {};
+        s2.a0 = static_cast<const uint8_t *>(ex->sh_down); s2.a_stride = 0; s2.rows = ex->d; s2.K = ex->f_shared;
+        s2.b_src = hs; s2.n_pos = T; s2.out = y_shared; s2.ldo = ex->d;
+        s = launch_grouped<DS4MOE_FMT_BF16, false>(s2, ex->d / GM_M, ct, st);
+        if (s != DS4MOE_OK) return s;
+    }
+    return DS4MOE_OK;
+}
+
+}  // namespace
+
+// =======================================================================================================
+extern "C" {
+
+const char *ds4moe_status_string(ds4moe_status s) {
+    switch (s) {
+    case DS4MOE_OK: return "ok";
+    case DS4MOE_EINVAL: return "invalid argument";
+    case DS4MOE_EUNSUPPORTED: return "unsupported format or shape";
+    case DS4MOE_ECUDA: return "CUDA error";
+    case DS4MOE_ENOWORKSPACE: return "workspace too small";
+    case DS4MOE_ETIMEOUT: return "device wait timed out";
+    case DS4MOE_EDEVICE: return "device-side data error";
+    }
+    return "unknown status";
+}
+
+size_t ds4moe_prepared_bytes(ds4moe_fmt fmt, int rows, int cols) {
+    if (!fmt_quant(fmt) || rows <= 0 || cols <= 0 || cols % QK) return 0;
+    return plane_layout(fmt, uint64_t(rows) * (cols / QK)).total;
+}
+
+ds4moe_status ds4moe_prepare(ds4moe_fmt fmt, const void *canonical, void *prepared, int rows, int cols, int n_mats,
+                             uint64_t prepared_stride, ds4moe_stream stream) {
+    (void)cudaGetLastError();  // report only errors raised by this call's launches
+    if (!fmt_quant(fmt)) return DS4MOE_EUNSUPPORTED;
+    if (!canonical || !prepared || rows <= 0 || cols <= 0 || cols % QK || n_mats < 0) return DS4MOE_EINVAL;
+    if (!aligned256(prepared) || prepared_stride % 256 || prepared_stride < ds4moe_prepared_bytes(fmt, rows, cols))
+        return DS4MOE_EINVAL;
+    if (n_mats == 0) return DS4MOE_OK;
+    const uint64_t nblk = uint64_t(rows) * (cols / QK);
+    const uint64_t total = nblk * n_mats;
+    const unsigned grid = unsigned((total + 255) / 256);
+    if (fmt == DS4MOE_FMT_IQ2X)
+        prepare_iq2x_kernel<<<grid, 256, 0, cs(stream)>>>(static_cast<const uint8_t *>(canonical),
+                                                          static_cast<uint8_t *>(prepared), nblk, n_mats,
+                                                          prepared_stride);
+    else
+        prepare_kquant_kernel<<<grid, 256, 0, cs(stream)>>>(static_cast<const uint8_t *>(canonical),
+                                                            static_cast<uint8_t *>(prepared), nblk, n_mats,
+                                                            prepared_stride, fmt);
+    DS4_CHECK_LAUNCH();
+    return DS4MOE_OK;
+}
+
+ds4moe_status ds4moe_dequant(ds4moe_fmt fmt, const void *prepared, const uint8_t *codebook, int rows, int cols,
+                             float *out, ds4moe_stream stream) {
+    (void)cudaGetLastError();  // report only errors raised by this call's launches
+    if (!fmt_quant(fmt)) return DS4MOE_EUNSUPPORTED;
+    if (!prepared || !out || rows <= 0 || cols <= 0 || cols % QK || !aligned256(prepared)) return DS4MOE_EINVAL;
+    if (fmt == DS4MOE_FMT_IQ2X && !codebook) return DS4MOE_EINVAL;
+    const uint8_t *p = static_cast<const uint8_t *>(prepared);
+    if (fmt == DS4MOE_FMT_IQ2X) {
+        const uint64_t n = uint64_t(rows) * (cols / 8);
+        dequant_iq2x_kernel<<<unsigned((n + 255) / 256), 256, 0, cs(stream)>>>(p, codebook, rows, cols, out);
+    } else {
+        const uint64_t n = uint64_t(rows) * (cols / (fmt == DS4MOE_FMT_Q2K ? 16 : 32));
+        dequant_kquant_kernel<<<unsigned((n + 255) / 256), 256, 0, cs(stream)>>>(p, rows, cols, fmt, out);
+    }
+    DS4_CHECK_LAUNCH();
+    return DS4MOE_OK;
+}
+
+size_t ds4moe_route_workspace_size(int T, int d, int E) {
+    (void)d;
+    if (T < 0 || E <= 0) return 0;
+    return a256(uint64_t(T > 0 ? T : 1) * E * 4);
+}
+
+ds4moe_status ds4moe_route(const void *x_bf16, int T, int d, const void *w_router_f16, const float *bias, int E,
+                           int k, int32_t *ids, float *weights, void *ws, size_t ws_bytes, ds4moe_stream stream) {
+    (void)cudaGetLastError();  // report only errors raised by this call's launches
+    if (T < 0 || d <= 0 || d % QK || E <= 0 || E > 1024 || k < 1 || k > E || k > 32) return DS4MOE_EINVAL;
+    if (T == 0) return DS4MOE_OK;
+    if (!x_bf16 || !w_router_f16 || !ids || !weights || !ws) return DS4MOE_EINVAL;
+    if (!aligned16(x_bf16) || !aligned16(w_router_f16)) return DS4MOE_EINVAL;
+    if (ws_bytes < ds4moe_route_workspace_size(T, d, E)) return DS4MOE_ENOWORKSPACE;
+    float *logits = static_cast<float *>(ws);
+    const __nv_bfloat16 *x = static_cast<const __nv_bfloat16 *>(x_bf16);
+    const __half *wr = static_cast<const __half *>(w_router_f16);
+    if (T <= ROUTE_SMALL_T) {
+        route_logits_small_kernel<<<(E + 1) / 2, 256, 0, cs(stream)>>>(x, T, d, wr, bias, E, logits);
+    } else {
+        route_logits_tiled_kernel<<<dim3((T + 63) / 64, (E + 63) / 64), 256, 0, cs(stream)>>>(x, T, d, wr, bias, E,
+                                                                                             logits);
+    }
+    DS4_CHECK_LAUNCH();
+    route_topk_kernel<<<(T + 7) / 8, 256, 0, cs(stream)>>>(logits, T, E, k, ids, weights);
+    DS4_CHECK_LAUNCH();
+    return DS4MOE_OK;
+}
+
+size_t ds4moe_workspace_size(const ds4moe_experts *ex, int T, int k) {
+    if (check_experts(ex) != DS4MOE_OK || T < 0 || k < 1 || k > ex->E) return 0;
+    const int TT = T > 0 ? T : 1;
+    uint64_t need = grouped_ws(ex, TT, k).total_decode;
+    if (decode_gemv_supported(ex, k)) {
+        const uint64_t dw = decode_ws(ex, k).total;
+        if (dw > need) need = dw;
+    }
+    return need;
+}
+
+ds4moe_status ds4moe_expert_ffn_decode(const ds4moe_experts *ex, const void *x_bf16, int B, const int32_t *ids,
+                                       const float *weights, int k, float *out, void *ws, size_t ws_bytes,
+                                       ds4moe_stream stream) {
+    (void)cudaGetLastError();  // report only errors raised by this call's launches
+    ds4moe_status s = check_experts(ex);
+    if (s != DS4MOE_OK) return s;
+    if (B < 0 || k < 1 || k > ex->E) return DS4MOE_EINVAL;
+    if (B == 0) return DS4MOE_OK;
+    if (!x_bf16 || !ids || !weights || !out || !ws || !aligned16(x_bf16) || !aligned256(ws) || !aligned16(out))
+        return DS4MOE_EINVAL;
+    if (ws_bytes < ds4moe_workspace_size(ex, B, k)) return DS4MOE_ENOWORKSPACE;
+    cudaStream_t st = cs(stream);
+    uint8_t *w8 = static_cast<uint8_t *>(ws);
+    if (B == 1 && decode_gemv_supported(ex, k)) {
+        s = ds4moe_decode_gateup(ex, x_bf16, ids, k, ws, ws_bytes, stream);
+        if (s != DS4MOE_OK) return s;
+        return ds4moe_decode_down(ex, ids, weights, k, out, ws, ws_bytes, stream);
+    }
+    // B > 1 (or a format without a GEMV kernel): grouped path, then combine
+    const GroupedWs W = grouped_ws(ex, B, k);
+    float *y_perm = reinterpret_cast<float *>(w8 + W.y_perm);
+    int32_t *inv = reinterpret_cast<int32_t *>(w8 + W.inv);
+    float *y_sh = ex->f_shared > 0 ? reinterpret_cast<float *>(w8 + W.y_shared) : nullptr;
+    s = run_grouped(ex, x_bf16, B, ids, weights, k, y_perm, inv, y_sh, w8, st);
+    if (s != DS4MOE_OK) return s;
+    return ds4moe_combine(y_perm, inv, y_sh, B, ex->d, k, out, stream);
+}
+
+ds4moe_status ds4moe_decode_gateup(const ds4moe_experts *ex, const void *x_bf16, const int32_t *ids, int k, void *ws,
+                                   size_t ws_bytes, ds4moe_stream stream) {
+    (void)cudaGetLastError();  // report only errors raised by this call's launches
+    ds4moe_status s = check_experts(ex);
+    if (s != DS4MOE_OK) return s;
+    if (k < 1 || k > ex->E) return DS4MOE_EINVAL;
+    if (!decode_gemv_supported(ex, k)) return DS4MOE_EUNSUPPORTED;
+    if (!x_bf16 || !ids || !ws || !aligned16(x_bf16) || !aligned256(ws)) return DS4MOE_EINVAL;
+    const DecodeWs W = decode_ws(ex, k);
+    if (ws_bytes < W.total) return DS4MOE_ENOWORKSPACE;
+    uint8_t *w8 = static_cast<uint8_t *>(ws);
+    const ExpertsDev D = to_dev(ex);
+    float *h = reinterpret_cast<float *>(w8 + W.h);
+    float *shp = reinterpret_cast<float *>(w8 + W.sh_part);
+    const __nv_bfloat16 *x = static_cast<const __nv_bfloat16 *>(x_bf16);
+    const int grid = num_sms();
+    cudaStream_t st = cs(stream);
+    cudaError_t err;
+    switch (ex->d / QK) {
+#define GU_CASE(V)                                                                                              \
+    case V:                                                                                                     \
+        if (!set_smem(decode_gateup_iq2x_kernel<V>, gu_smem_bytes(ex->d))) return DS4MOE_ECUDA;                 \
+        err = launch_pdl(decode_gateup_iq2x_kernel<V>, dim3(grid), dim3(GU_THREADS), size_t(gu_smem_bytes(ex->d)), \
+                         st, D, x, ids, k, h, shp);                                                             \
+        break;
+        GU_CASE(1) GU_CASE(2) GU_CASE(4) GU_CASE(8) GU_CASE(16)
+#undef GU_CASE
+    default: return DS4MOE_EUNSUPPORTED;
+    }
+    if (err != cudaSuccess) {
+        (void)cudaGetLastError();
+        return DS4MOE_ECUDA;
+    }
+    return DS4MOE_OK;
+}
+
+ds4moe_status ds4moe_decode_down(const ds4moe_experts *ex, const int32_t *ids, const float *weights, int k, float *out,
+                                 void *ws, size_t ws_bytes, ds4moe_stream stream) {
+    (void)cudaGetLastError();  // report only errors raised by this call's launches
+    ds4moe_status s = check_experts(ex);
+    if (s != DS4MOE_OK) return s;
+    if (k < 1 || k > ex->E) return DS4MOE_EINVAL;
+    if (!decode_gemv_supported(ex, k)) return DS4MOE_EUNSUPPORTED;
+    if (!ids || !weights || !out || !ws || !aligned16(out) || !aligned256(ws)) return DS4MOE_EINVAL;
+    const DecodeWs W = decode_ws(ex, k);
+    if (ws_bytes < W.total) return DS4MOE_ENOWORKSPACE;
+    uint8_t *w8 = static_cast<uint8_t *>(ws);
+    const ExpertsDev D = to_dev(ex);
+    const float *h = reinterpret_cast<const float *>(w8 + W.h);
+    const float *shp = reinterpret_cast<const float *>(w8 + W.sh_part);
+    const int grid = num_sms();
+    const int wpl = ex->f <= 512 ? 1 : ex->f / 512;
+    const DownSmem L = down_smem_layout(k, wpl, ex->f_shared);
+    cudaStream_t st = cs(stream);
+    cudaError_t err;
+    switch (wpl) {
+#define DN_CASE(V)                                                                                               \
+    case V:                                                                                                      \
+        if (!set_smem(decode_down_q2k_kernel<V>, L.total)) return DS4MOE_ECUDA;                                  \
+        err = launch_pdl(decode_down_q2k_kernel<V>, dim3(grid), dim3(DN_THREADS), size_t(L.total), st, D, h, shp, \
+                         W.nch, ids, weights, k, out);                                                          \
+        break;
+        DN_CASE(1) DN_CASE(2) DN_CASE(4) DN_CASE(8)
+#undef DN_CASE
+    default: return DS4MOE_EUNSUPPORTED;
+    }
+    if (err != cudaSuccess) {
+        (void)cudaGetLastError();
+        return DS4MOE_ECUDA;
+    }
+    return DS4MOE_OK;
+}
+
+ds4moe_status ds4moe_expert_ffn_grouped(const ds4moe_experts *ex, const void *x_bf16, int T, const int32_t *ids,
+                                        const float *weights, int k, float *y_perm, int32_t *inv_perm,
+                                        float *y_shared, void *ws, size_t ws_bytes, ds4moe_stream stream) {
+    (void)cudaGetLastError();  // report only errors raised by this call's launches
+    ds4moe_status s = check_experts(ex);
+    if (s != DS4MOE_OK) return s;
+    if (T < 0 || k < 1 || k > ex->E) return DS4MOE_EINVAL;
+    if (T == 0) return DS4MOE_OK;
+    if (!x_bf16 || !ids || !weights || !y_perm || !inv_perm || !ws || !aligned16(x_bf16) || !aligned256(ws) ||
+        !aligned16(y_perm))
+        return DS4MOE_EINVAL;
+    if (ex->f_shared > 0 && (!y_shared || !aligned16(y_shared))) return DS4MOE_EINVAL;
+    if (ws_bytes < grouped_ws(ex, T, k).total_grouped) return DS4MOE_ENOWORKSPACE;
+    return run_grouped(ex, x_bf16, T, ids, weights, k, y_perm, inv_perm, ex->f_shared > 0 ? y_shared : nullptr,
+                       static_cast<uint8_t *>(ws), cs(stream));
+}
+
+ds4moe_status ds4moe_combine(const float *y_perm, const int32_t *inv_perm, const float *y_shared, int T, int d, int k,
+                             float *out, ds4moe_stream stream) {
+    if (T < 0 || d <= 0 || d % 4 || k < 1) return DS4MOE_EINVAL;
+    if (T == 0) return DS4MOE_OK;
+    if (!y_perm || !inv_perm || !out || !aligned16(y_perm) || !aligned16(out)) return DS4MOE_EINVAL;
+    if (y_shared && !aligned16(y_shared)) return DS4MOE_EINVAL;
+    const uint64_t total = uint64_t(T) * (d / 4);
+    const unsigned grid = unsigned(std::min<uint64_t>((total + 255) / 256, uint64_t(num_sms()) * 16));
+    combine_kernel<<<grid, 256, 0, cs(stream)>>>(y_perm, inv_perm, y_shared, T, d, k, out);
+    DS4_CHECK_LAUNCH();
+    return DS4MOE_OK;
+}
+
+ds4moe_status ds4moe_last_device_error(ds4moe_stream stream, int32_t *code) {
+    if (!code) return DS4MOE_EINVAL;
+    if (cudaStreamSynchronize(cs(stream)) != cudaSuccess) return DS4MOE_ECUDA;
+    int32_t v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(v)) != cudaSuccess) return DS4MOE_ECUDA;
+    if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)) != cudaSuccess) return DS4MOE_ECUDA;
+    *code = v;
+    return DS4MOE_OK;
+}
+
+}  // extern "C"

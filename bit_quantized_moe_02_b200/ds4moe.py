@@ -1,0 +1,250 @@
+"""ctypes binding of libds4moe.so (include/ds4moe.h), argument marshalling only.
+
+Tensors are torch CUDA tensors; every call runs on the current torch stream.
+Nothing here computes any part of the layer: each step runs in the library's
+kernels, and a missing library raises instead of falling back.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import numpy as np
+import torch
+
+from . import synth
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libds4moe.so")
+
+FMT = {"iq2x": 0, "q2k": 1, "q4k": 2, "bf16": 3}
+STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported", 3: "CUDA error", 4: "workspace too small",
+          5: "device wait timed out", 6: "device-side data error"}
+
+EXPORTS = ["ds4moe_status_string", "ds4moe_prepared_bytes", "ds4moe_prepare", "ds4moe_dequant",
+           "ds4moe_route_workspace_size", "ds4moe_route", "ds4moe_workspace_size", "ds4moe_expert_ffn_decode",
+           "ds4moe_expert_ffn_grouped", "ds4moe_combine", "ds4moe_last_device_error", "ds4moe_decode_gateup",
+           "ds4moe_decode_down"]
+
+
+class Ds4moeError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__("%s failed: %s (%d)" % (what, STATUS.get(code, "?"), code))
+        self.code = code
+
+
+class Experts(ctypes.Structure):
+    _fields_ = [("d", ctypes.c_int32), ("f", ctypes.c_int32), ("E", ctypes.c_int32), ("f_shared", ctypes.c_int32),
+                ("fmt_gate", ctypes.c_int32), ("fmt_up", ctypes.c_int32), ("fmt_down", ctypes.c_int32),
+                ("gate", ctypes.c_void_p), ("up", ctypes.c_void_p), ("down", ctypes.c_void_p),
+                ("gate_stride", ctypes.c_uint64), ("up_stride", ctypes.c_uint64), ("down_stride", ctypes.c_uint64),
+                ("codebook", ctypes.c_void_p),
+                ("sh_gate", ctypes.c_void_p), ("sh_up", ctypes.c_void_p), ("sh_down", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def lib():
+    """Load the library (raises if it was not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError("libds4moe.so is missing: run `python -m bit_quantized_moe_02_b200.build`")
+        l = ctypes.CDLL(LIB_PATH)
+        vp, i32, u64, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint64, ctypes.c_size_t
+        l.ds4moe_status_string.restype = ctypes.c_char_p
+        l.ds4moe_status_string.argtypes = [i32]
+        l.ds4moe_prepared_bytes.restype = sz
+        l.ds4moe_prepared_bytes.argtypes = [i32, i32, i32]
+        l.ds4moe_prepare.argtypes = [i32, vp, vp, i32, i32, i32, u64, vp]
+        l.ds4moe_dequant.argtypes = [i32, vp, vp, i32, i32, vp, vp]
+        l.ds4moe_route_workspace_size.restype = sz
+        l.ds4moe_route_workspace_size.argtypes = [i32, i32, i32]
+        l.ds4moe_route.argtypes = [vp, i32, i32, vp, vp, i32, i32, vp, vp, vp, sz, vp]
+        l.ds4moe_workspace_size.restype = sz
+        l.ds4moe_workspace_size.argtypes = [ctypes.POINTER(Experts), i32, i32]
+        l.ds4moe_expert_ffn_decode.argtypes = [ctypes.POINTER(Experts), vp, i32, vp, vp, i32, vp, vp, sz, vp]
+        l.ds4moe_expert_ffn_grouped.argtypes = [ctypes.POINTER(Experts), vp, i32, vp, vp, i32, vp, vp, vp, vp, sz,
+                                                vp]
+        l.ds4moe_combine.argtypes = [vp, vp, vp, i32, i32, i32, vp, vp]
+        l.ds4moe_last_device_error.argtypes = [vp, ctypes.POINTER(ctypes.c_int32)]
+        l.ds4moe_decode_gateup.argtypes = [ctypes.POINTER(Experts), vp, vp, i32, vp, sz, vp]
+        l.ds4moe_decode_down.argtypes = [ctypes.POINTER(Experts), vp, vp, i32, vp, vp, sz, vp]
+        _lib = l
+    return _lib
+
+
+def _check(code: int, what: str) -> None:
+    if code != 0:
+        raise Ds4moeError(code, what)
+
+
+def _p(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+# ---- thin wrappers, one per C entry point ----------------------------------------------------------------
+
+def prepared_bytes(fmt: str, rows: int, cols: int) -> int:
+    return int(lib().ds4moe_prepared_bytes(FMT[fmt], rows, cols))
+
+
+def prepare(fmt: str, canonical: torch.Tensor, rows: int, cols: int, n_mats: int,
+            out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    stride = (prepared_bytes(fmt, rows, cols) + 255) // 256 * 256
+    if out is None:
+        out = torch.empty(stride * max(n_mats, 1), dtype=torch.uint8, device=canonical.device)
+    _check(lib().ds4moe_prepare(FMT[fmt], _p(canonical), _p(out), rows, cols, n_mats, stride, _stream()), "prepare")
+    return out
+
+
+def dequant(fmt: str, prepared: torch.Tensor, codebook: Optional[torch.Tensor], rows: int, cols: int) -> torch.Tensor:
+    out = torch.empty((rows, cols), dtype=torch.float32, device=prepared.device)
+    _check(lib().ds4moe_dequant(FMT[fmt], _p(prepared), _p(codebook), rows, cols, _p(out), _stream()), "dequant")
+    return out
+
+
+def route(x: torch.Tensor, wr: torch.Tensor, bias: Optional[torch.Tensor], k: int, ws: Optional[torch.Tensor] = None,
+          ids: Optional[torch.Tensor] = None, weights: Optional[torch.Tensor] = None):
+    T, d = x.shape
+    E = wr.shape[0]
+    need = int(lib().ds4moe_route_workspace_size(T, d, E))
+    if ws is None or ws.numel() < need:
+        ws = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
+    ids = torch.empty((T, k), dtype=torch.int32, device=x.device) if ids is None else ids
+    weights = torch.empty((T, k), dtype=torch.float32, device=x.device) if weights is None else weights
+    _check(lib().ds4moe_route(_p(x), T, d, _p(wr), _p(bias), E, k, _p(ids), _p(weights), _p(ws), ws.numel(),
+                              _stream()), "route")
+    return ids, weights
+
+
+def workspace_size(ex: Experts, T: int, k: int) -> int:
+    return int(lib().ds4moe_workspace_size(ctypes.byref(ex), T, k))
+
+
+def expert_ffn_decode(ex: Experts, x: torch.Tensor, ids: torch.Tensor, weights: torch.Tensor, ws: torch.Tensor,
+                      out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    B, k = ids.shape
+    out = torch.empty((B, ex.d), dtype=torch.float32, device=x.device) if out is None else out
+    _check(lib().ds4moe_expert_ffn_decode(ctypes.byref(ex), _p(x), B, _p(ids), _p(weights), k, _p(out), _p(ws),
+                                          ws.numel(), _stream()), "expert_ffn_decode")
+    return out
+
+
+def decode_gateup(ex: Experts, x: torch.Tensor, ids: torch.Tensor, ws: torch.Tensor) -> None:
+    _check(lib().ds4moe_decode_gateup(ctypes.byref(ex), _p(x), _p(ids), ids.shape[-1], _p(ws), ws.numel(), _stream()),
+           "decode_gateup")
+
+
+def decode_down(ex: Experts, ids: torch.Tensor, weights: torch.Tensor, ws: torch.Tensor, out: torch.Tensor) -> None:
+    _check(lib().ds4moe_decode_down(ctypes.byref(ex), _p(ids), _p(weights), ids.shape[-1], _p(out), _p(ws),
+                                    ws.numel(), _stream()), "decode_down")
+
+
+def expert_ffn_grouped(ex: Experts, x: torch.Tensor, ids: torch.Tensor, weights: torch.Tensor, ws: torch.Tensor,
+                       y_perm: torch.Tensor, inv_perm: torch.Tensor, y_shared: Optional[torch.Tensor]) -> None:
+    T, k = ids.shape
+    _check(lib().ds4moe_expert_ffn_grouped(ctypes.byref(ex), _p(x), T, _p(ids), _p(weights), k, _p(y_perm),
+                                           _p(inv_perm), _p(y_shared), _p(ws), ws.numel(), _stream()),
+           "expert_ffn_grouped")
+
+
+def combine(y_perm: torch.Tensor, inv_perm: torch.Tensor, y_shared: Optional[torch.Tensor], T: int, d: int, k: int,
+            out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    out = torch.empty((T, d), dtype=torch.float32, device=y_perm.device) if out is None else out
+    _check(lib().ds4moe_combine(_p(y_perm), _p(inv_perm), _p(y_shared), T, d, k, _p(out), _stream()), "combine")
+    return out
+
+
+def last_device_error() -> int:
+    code = ctypes.c_int32(0)
+    _check(lib().ds4moe_last_device_error(_stream(), ctypes.byref(code)), "last_device_error")
+    return int(code.value)
+
+
+# ---- a layer held on the device ------------------------------------------------------------------------------
+
+class DeviceLayer:
+    """One MoE FFN layer resident in HBM: prepared expert planes, codebook, router, shared expert.
+
+    ``forward(x)`` runs route -> experts -> combine for any number of tokens: T = 1 takes the decode GEMV path,
+    larger T the permuted grouped path.  All buffers, including the workspace, are allocated here once.
+    """
+
+    def __init__(self, host: "synth.Layer", device="cuda", max_tokens: int = 1):
+        s = host.shape
+        self.shape = s
+        self.device = torch.device(device)
+        dev = self.device
+
+        def up(a):
+            return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+        self.wr = up(host.wr).view(torch.float16)
+        self.bias = up(host.bias) if np.any(host.bias != 0) else None
+        self.codebook = up(host.grid.reshape(-1))
+        self.planes = {}
+        strides = {}
+        for which, fmt, rows, cols in (("gate", s.fmt_gate, s.f, s.d), ("up", s.fmt_up, s.f, s.d),
+                                       ("down", s.fmt_down, s.d, s.f)):
+            stride = (prepared_bytes(fmt, rows, cols) + 255) // 256 * 256
+            buf = torch.empty(stride * s.E, dtype=torch.uint8, device=dev)
+            chunk = 16  # experts uploaded per canonical staging copy
+            for e0 in range(0, s.E, chunk):
+                e1 = min(s.E, e0 + chunk)
+                canon = up(np.stack([host.expert(which, e) for e in range(e0, e1)]))
+                prepare(fmt, canon, rows, cols, e1 - e0, out=buf[e0 * stride:])
+                del canon
+            self.planes[which] = buf
+            strides[which] = stride
+        host.drop_cache()
+        self.sh = [None if a is None else up(a).view(torch.bfloat16) for a in (host.sh_gate, host.sh_up,
+                                                                                host.sh_down)]
+        fs = s.f_shared if self.sh[0] is not None else 0
+        self.ex = Experts(s.d, s.f, s.E, fs, FMT[s.fmt_gate], FMT[s.fmt_up], FMT[s.fmt_down],
+                          self.planes["gate"].data_ptr(), self.planes["up"].data_ptr(),
+                          self.planes["down"].data_ptr(), strides["gate"], strides["up"], strides["down"],
+                          self.codebook.data_ptr(),
+                          self.sh[0].data_ptr() if fs else None, self.sh[1].data_ptr() if fs else None,
+                          self.sh[2].data_ptr() if fs else None)
+        self.max_tokens = 0
+        self.reserve(max_tokens)
+
+    def reserve(self, T: int) -> None:
+        if T <= self.max_tokens:
+            return
+        s = self.shape
+        need = max(workspace_size(self.ex, T, s.k), 1)
+        self.ws = torch.empty(need, dtype=torch.uint8, device=self.device)
+        self.route_ws = torch.empty(max(int(lib().ds4moe_route_workspace_size(T, s.d, s.E)), 1), dtype=torch.uint8,
+                                    device=self.device)
+        self.max_tokens = T
+
+    def route(self, x: torch.Tensor):
+        return route(x, self.wr, self.bias, self.shape.k, ws=self.route_ws)
+
+    def forward(self, x: torch.Tensor, out: Optional[torch.Tensor] = None, return_routing: bool = False):
+        T = x.shape[0]
+        self.reserve(T)
+        ids, w = self.route(x)
+        out = expert_ffn_decode(self.ex, x, ids, w, self.ws, out=out)
+        return (out, ids, w) if return_routing else out
+
+    def forward_grouped(self, x: torch.Tensor):
+        """Prefill entry: grouped experts then combine (returns out, ids, weights, y_perm, inv_perm)."""
+        s = self.shape
+        T = x.shape[0]
+        self.reserve(T)
+        ids, w = self.route(x)
+        y_perm = torch.empty((T * s.k, s.d), dtype=torch.float32, device=x.device)
+        inv = torch.empty(T * s.k, dtype=torch.int32, device=x.device)
+        ys = torch.empty((T, s.d), dtype=torch.float32, device=x.device) if self.ex.f_shared else None
+        expert_ffn_grouped(self.ex, x, ids, w, self.ws, y_perm, inv, ys)
+        out = combine(y_perm, inv, ys, T, s.d, s.k)
+        return out, ids, w, y_perm, inv

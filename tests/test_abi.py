@@ -1,0 +1,79 @@
+"""The C-ABI library loads without a GPU, exports every symbol the header declares, and its host-side checks
+reject bad arguments before launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from bit_quantized_moe_02_b200 import ds4moe
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def header_symbols():
+    src = open(os.path.join(ROOT, "include", "ds4moe.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(ds4moe_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_library_exports_every_header_symbol():
+    lib = ds4moe.lib()
+    syms = header_symbols()
+    assert len(syms) >= 13
+    for s in syms:
+        assert hasattr(lib, s), s
+    assert sorted(ds4moe.EXPORTS) == [s for s in syms if s in ds4moe.EXPORTS]
+
+
+def test_status_strings():
+    lib = ds4moe.lib()
+    for code in range(7):
+        assert lib.ds4moe_status_string(code)
+    assert lib.ds4moe_status_string(99) == b"unknown status"
+
+
+def test_prepared_bytes_layout():
+    # planes rounded to 256 B: IQ2X 32+32+4+2 B per block, Q2K 64+16+4, Q4K 128+12+4
+    def r(x):
+        return (x + 255) // 256 * 256
+    for rows, cols in ((1, 256), (512, 256), (2048, 4096), (4096, 2048), (3, 768)):
+        n = rows * cols // 256
+        assert ds4moe.prepared_bytes("iq2x", rows, cols) == r(32 * n) * 2 + r(4 * n) + r(2 * n)
+        assert ds4moe.prepared_bytes("q2k", rows, cols) == r(64 * n) + r(16 * n) + r(4 * n)
+        assert ds4moe.prepared_bytes("q4k", rows, cols) == r(128 * n) + r(12 * n) + r(4 * n)
+    assert ds4moe.prepared_bytes("iq2x", 4, 100) == 0
+    assert ds4moe.prepared_bytes("bf16", 4, 256) == 0
+
+
+def test_host_side_argument_checks():
+    lib = ds4moe.lib()
+    vp = ctypes.c_void_p
+    fake = vp(1 << 20)  # never dereferenced: every call below fails its host checks first
+    assert lib.ds4moe_prepare(0, None, fake, 4, 256, 1, 4096, None) == 1
+    assert lib.ds4moe_prepare(0, fake, fake, 4, 100, 1, 4096, None) == 1
+    assert lib.ds4moe_prepare(3, fake, fake, 4, 256, 1, 4096, None) == 2
+    assert lib.ds4moe_prepare(0, fake, vp((1 << 20) + 16), 4, 256, 1, 4096, None) == 1  # unaligned planes
+    assert lib.ds4moe_prepare(0, fake, fake, 4, 256, 1, 256, None) == 1  # stride below prepared size
+    assert lib.ds4moe_route(fake, 1, 256, fake, None, 8, 9, fake, fake, fake, 1 << 20, None) == 1  # k > E
+    assert lib.ds4moe_route(fake, 1, 256, fake, None, 2048, 2, fake, fake, fake, 1 << 20, None) == 1  # E > 1024
+    assert lib.ds4moe_route(fake, 1, 256, fake, None, 8, 2, fake, fake, fake, 4, None) == 4  # workspace
+    assert lib.ds4moe_route(None, 0, 256, None, None, 8, 2, None, None, None, 0, None) == 0  # T = 0: no-op
+    assert lib.ds4moe_combine(fake, fake, None, 1, 10, 2, fake, None) == 1  # d % 4
+    ex = ds4moe.Experts(256, 512, 8, 0, 0, 0, 1, 1 << 20, 1 << 21, 1 << 22, 1 << 16, 1 << 16, 1 << 16, 1 << 23,
+                        None, None, None)
+    assert lib.ds4moe_workspace_size(ctypes.byref(ex), 1, 2) > 0
+    bad = ds4moe.Experts(*[getattr(ex, f) for f, _ in ds4moe.Experts._fields_])
+    bad.fmt_up = 2
+    assert lib.ds4moe_workspace_size(ctypes.byref(bad), 1, 2) == 0
+    assert lib.ds4moe_expert_ffn_decode(ctypes.byref(bad), fake, 1, fake, fake, 2, fake, fake, 1 << 30, None) == 2
+    assert lib.ds4moe_expert_ffn_decode(ctypes.byref(ex), fake, 1, fake, fake, 2, fake, fake, 16, None) == 4
+    bad.fmt_up = 0
+    bad.gate_stride = 1000
+    assert lib.ds4moe_expert_ffn_grouped(ctypes.byref(bad), fake, 4, fake, fake, 2, fake, fake, None, fake, 1 << 30,
+                                         None) == 1
+    bad.gate_stride = 1 << 16
+    bad.f_shared = 256  # shared expert without weights
+    assert lib.ds4moe_expert_ffn_grouped(ctypes.byref(bad), fake, 4, fake, fake, 2, fake, fake, None, fake, 1 << 30,
+                                         None) == 1
+    assert lib.ds4moe_last_device_error(None, None) == 1
