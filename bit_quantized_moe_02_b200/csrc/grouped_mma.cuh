@@ -122,11 +122,18 @@ __device__ __forceinline__ int q4k_field(uint32_t s0, uint32_t s1, uint32_t s2, 
     return int(((lo >> pos) | (uint64_t(s2) << (64 - pos))) & 63u);
 }
 
-// Dequantize 32 weights into 4 uint4 (8 fp16 each, consecutive k).
-template <int AFMT>
-__device__ __forceinline__ void a_dequant(const APack &pk, const uint8_t *tbl, int k0, uint4 (&o)[4]) {
+// Dequantize 32 weights into 4 uint4 (8 fp16 each, consecutive k).  The IQ2X codebook table holds entry i
+// at tbl + i * TSTRIDE (8 fp16 values); bf16 rows are converted, setting *inf if a value leaves fp16 range.
+template <int AFMT, int TSTRIDE = 16>
+__device__ __forceinline__ void a_dequant(const APack &pk, const uint8_t *tbl, int k0, uint4 (&o)[4],
+                                          bool &inf) {
     constexpr uint32_t M = 0x80008000u;
-    if constexpr (AFMT == DS4MOE_FMT_IQ2X) {
+    if constexpr (AFMT == DS4MOE_FMT_BF16) {
+#pragma unroll
+        for (int j = 0; j < 4; j++)
+            o[j] = make_uint4(bf16x2_to_f16x2(pk.w[4 * j], inf), bf16x2_to_f16x2(pk.w[4 * j + 1], inf),
+                              bf16x2_to_f16x2(pk.w[4 * j + 2], inf), bf16x2_to_f16x2(pk.w[4 * j + 3], inf));
+    } else if constexpr (AFMT == DS4MOE_FMT_IQ2X) {
         const float dv = half_bits_to_float(uint16_t(pk.w[3]));
         const float s = float((pk.w[2] >> (4 * pk.w[4])) & 15u);
         const __half2 D2 = __float2half2_rn((dv * (0.5f + s)) * 0.25f);
@@ -134,7 +141,7 @@ __device__ __forceinline__ void a_dequant(const APack &pk, const uint8_t *tbl, i
 #pragma unroll
         for (int j = 0; j < 4; j++) {
             const uint32_t ib = (pk.w[0] >> (8 * j)) & 0xFFu;
-            const uint4 cb = *reinterpret_cast<const uint4 *>(tbl + ib * 16);
+            const uint4 cb = *reinterpret_cast<const uint4 *>(tbl + ib * TSTRIDE);
             const uint32_t Wj = W << (4 * j);
             o[j].x = half2_as_u32(__hmul2(u32_as_half2(cb.x ^ (Wj & M)), D2));
             o[j].y = half2_as_u32(__hmul2(u32_as_half2(cb.y ^ ((Wj << 1) & M)), D2));
@@ -266,20 +273,12 @@ __global__ void __launch_bounds__(GM_THREADS) grouped_mma_kernel(GroupedArgs a) 
     };
     auto store_a = [&](const APack &pk, int kc, int stage) {
         uint8_t *dst = As + stage * GM_A_BYTES;
-        if constexpr (AFMT == DS4MOE_FMT_BF16) {
-            bool inf = false;
+        uint4 o[4];
+        bool inf = false;
+        a_dequant<AFMT>(pk, tbl, kc * GM_K + hh * 32, o, inf);
 #pragma unroll
-            for (int j = 0; j < 4; j++)
-                *reinterpret_cast<uint4 *>(dst + swz(R, hh * 4 + j)) =
-                    make_uint4(bf16x2_to_f16x2(pk.w[4 * j], inf), bf16x2_to_f16x2(pk.w[4 * j + 1], inf),
-                               bf16x2_to_f16x2(pk.w[4 * j + 2], inf), bf16x2_to_f16x2(pk.w[4 * j + 3], inf));
-            if (inf) set_device_error(DS4MOE_EDEVICE);
-        } else {
-            uint4 o[4];
-            a_dequant<AFMT>(pk, tbl, kc * GM_K + hh * 32, o);
-#pragma unroll
-            for (int j = 0; j < 4; j++) *reinterpret_cast<uint4 *>(dst + swz(R, hh * 4 + j)) = o[j];
-        }
+        for (int j = 0; j < 4; j++) *reinterpret_cast<uint4 *>(dst + swz(R, hh * 4 + j)) = o[j];
+        if (inf) set_device_error(DS4MOE_EDEVICE);
     };
 
     float acc[2][4][4];
