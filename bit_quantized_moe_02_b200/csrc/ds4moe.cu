@@ -243,6 +243,37 @@ ds4moe_status run_grouped(const ds4moe_experts *ex, const void *x, int T, const 
     return DS4MOE_OK;
 }
 
+// ---- scratch for the allocation-free decode entry point ------------------------------------------------
+//
+// Some callers cannot hand the library a workspace: code that must not call cudaMalloc at all
+// (an engine whose memory planner already owns all of HBM and forbids any further allocation, a
+// plugin host that exposes no allocator).  ds4moe_expert_ffn_decode_noalloc serves them from this
+// fixed array instead.  Every GPU that loads the library holds it until the process exits.
+constexpr size_t NOALLOC_SCRATCH_BYTES = size_t(1) << 20;  // 1 MiB
+static __device__ __align__(256) uint8_t g_noalloc_scratch[NOALLOC_SCRATCH_BYTES];
+
+// Device address of g_noalloc_scratch per device.  The host-side symbol is only a stand-in, so the
+// address is looked up once per device, with that device current, and cached.
+void *noalloc_scratch_on_current_device(ds4moe_status *st) {
+    static void *cache[64] = {nullptr};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        *st = DS4MOE_ECUDA;
+        return nullptr;
+    }
+    if (!cache[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+            (void)cudaGetLastError();
+            *st = DS4MOE_ECUDA;
+            return nullptr;
+        }
+        cache[dev] = p;
+    }
+    *st = DS4MOE_OK;
+    return cache[dev];
+}
+
 }  // namespace
 
 // =======================================================================================================
@@ -446,6 +477,24 @@ ds4moe_status ds4moe_decode_down(const ds4moe_experts *ex, const int32_t *ids, c
         return DS4MOE_ECUDA;
     }
     return DS4MOE_OK;
+}
+
+ds4moe_status ds4moe_expert_ffn_decode_noalloc(const ds4moe_experts *ex, const void *x_bf16, const int32_t *ids,
+                                               const float *weights, int k, float *out, ds4moe_stream stream) {
+    (void)cudaGetLastError();  // report only errors raised by this call's launches
+    ds4moe_status s = check_experts(ex);
+    if (s != DS4MOE_OK) return s;
+    if (k < 1 || k > ex->E) return DS4MOE_EINVAL;
+    if (!decode_gemv_supported(ex, k)) return DS4MOE_EUNSUPPORTED;
+    if (!x_bf16 || !ids || !weights || !out || !aligned16(x_bf16) || !aligned16(out)) return DS4MOE_EINVAL;
+    const uint64_t need = decode_ws(ex, k).total;
+    if (need > NOALLOC_SCRATCH_BYTES) return DS4MOE_ENOWORKSPACE;  // layer too large for the fixed scratch
+    void *scratch = noalloc_scratch_on_current_device(&s);
+    if (s != DS4MOE_OK) return s;
+    // the gate/up kernel overwrites every scratch word the down kernel reads: nothing to clear
+    s = ds4moe_decode_gateup(ex, x_bf16, ids, k, scratch, NOALLOC_SCRATCH_BYTES, stream);
+    if (s != DS4MOE_OK) return s;
+    return ds4moe_decode_down(ex, ids, weights, k, out, scratch, NOALLOC_SCRATCH_BYTES, stream);
 }
 
 ds4moe_status ds4moe_expert_ffn_grouped(const ds4moe_experts *ex, const void *x_bf16, int T, const int32_t *ids,

@@ -25,7 +25,7 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported", 3: "CUDA error", 4: 
 EXPORTS = ["ds4moe_status_string", "ds4moe_prepared_bytes", "ds4moe_prepare", "ds4moe_dequant",
            "ds4moe_route_workspace_size", "ds4moe_route", "ds4moe_workspace_size", "ds4moe_expert_ffn_decode",
            "ds4moe_expert_ffn_grouped", "ds4moe_combine", "ds4moe_last_device_error", "ds4moe_decode_gateup",
-           "ds4moe_decode_down"]
+           "ds4moe_decode_down", "ds4moe_expert_ffn_decode_noalloc"]
 
 
 class Ds4moeError(RuntimeError):
@@ -72,6 +72,7 @@ def lib():
         l.ds4moe_last_device_error.argtypes = [vp, ctypes.POINTER(ctypes.c_int32)]
         l.ds4moe_decode_gateup.argtypes = [ctypes.POINTER(Experts), vp, vp, i32, vp, sz, vp]
         l.ds4moe_decode_down.argtypes = [ctypes.POINTER(Experts), vp, vp, i32, vp, vp, sz, vp]
+        l.ds4moe_expert_ffn_decode_noalloc.argtypes = [ctypes.POINTER(Experts), vp, vp, vp, i32, vp, vp]
         _lib = l
     return _lib
 
@@ -145,6 +146,15 @@ def decode_gateup(ex: Experts, x: torch.Tensor, ids: torch.Tensor, ws: torch.Ten
 def decode_down(ex: Experts, ids: torch.Tensor, weights: torch.Tensor, ws: torch.Tensor, out: torch.Tensor) -> None:
     _check(lib().ds4moe_decode_down(ctypes.byref(ex), _p(ids), _p(weights), ids.shape[-1], _p(out), _p(ws),
                                     ws.numel(), _stream()), "decode_down")
+
+
+def expert_ffn_decode_noalloc(ex: Experts, x: torch.Tensor, ids: torch.Tensor, weights: torch.Tensor,
+                              out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """B = 1 decode served from the library's fixed scratch array (no workspace argument)."""
+    out = torch.empty((1, ex.d), dtype=torch.float32, device=x.device) if out is None else out
+    _check(lib().ds4moe_expert_ffn_decode_noalloc(ctypes.byref(ex), _p(x), _p(ids), _p(weights), ids.shape[-1],
+                                                  _p(out), _stream()), "expert_ffn_decode_noalloc")
+    return out
 
 
 def expert_ffn_grouped(ex: Experts, x: torch.Tensor, ids: torch.Tensor, weights: torch.Tensor, ws: torch.Tensor,

@@ -177,6 +177,24 @@ ds4moe_status ds4moe_decode_gateup(const ds4moe_experts *ex, const void *x_bf16,
 ds4moe_status ds4moe_decode_down(const ds4moe_experts *ex, const int32_t *ids, const float *weights, int k,
                                  float *out, void *ws, size_t ws_bytes, ds4moe_stream stream);
 
+/* Single-token decode without a caller workspace, for callers that cannot
+ * allocate device memory at all: an engine whose memory planner has taken all
+ * of HBM and forbids further allocation, or a plugin host that exposes no
+ * allocator.  The paper has no counterpart: this is a library convenience.
+ * Same computation and arguments as ds4moe_expert_ffn_decode with B = 1 (and
+ * the same format limits as ds4moe_decode_gateup), but the scratch comes from
+ * a 1 MiB array compiled into the library, which every GPU that loads the
+ * library holds until the process exits.  Layers whose decode scratch
+ * (4 * (k*f + 2*f_shared*ceil(d/1024)) bytes, rounded) exceeds 1 MiB are
+ * rejected with DS4MOE_ENOWORKSPACE.  Nothing is allocated: no cudaMalloc, no
+ * cudaFree.  The first call on a device looks up the array's device address
+ * (once per device, with that device current); make that first call before
+ * any stream capture.  All calls share the one array, which keeps the last
+ * call's contents: calls whose kernels overlap on the GPU (other streams,
+ * other threads) race on it, so serialize them. */
+ds4moe_status ds4moe_expert_ffn_decode_noalloc(const ds4moe_experts *ex, const void *x_bf16, const int32_t *ids,
+                                               const float *weights, int k, float *out, ds4moe_stream stream);
+
 /* Prefill / many tokens.  Permutes the T*k (token, slot) pairs by expert id
  * (stable: increasing token, then slot), runs the grouped dequantize-GEMM
  * SwiGLU experts and writes
