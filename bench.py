@@ -365,6 +365,36 @@ def run_prefill(args, ds4moe, torch, stream, tf, tf_sus, peak_kind):
             "frac_of_bf16_peak": flops / (ms / 1e3) / 1e12 / tf, "peak_tflops": tf, "peak_kind": peak_kind}
 
 
+def run_profile_case(args):
+    """Small case for ncu captures, same kernels and shapes as the benchmark but fewer experts resident:
+    decode layer d=4096, f=2048, k=8, shared 2048 with E=16 experts (the 8 a token uses stream 56 MB of packed
+    weights + 50 MB of shared weights per pass, more than L2), 16 eager B=1 passes; optionally a prefill of
+    T tokens on E=64 experts (T=1024, k=8 keeps the prefill workload's 128 tokens per expert on average)."""
+    import dataclasses
+
+    import torch
+    from bit_quantized_moe_02_b200 import ds4moe
+    base = synth.WORKLOADS["decode"]
+    wl = dataclasses.replace(base, shape=dataclasses.replace(base.shape, E=16))
+    D = ds4moe.DeviceLayer(synth.make_layer(wl), max_tokens=1)
+    xs = torch.from_numpy(synth.activations(wl, 16, stream=3)).cuda().view(torch.bfloat16)
+    for i in range(16):
+        D.forward(xs[i:i + 1])
+    torch.cuda.synchronize()
+    if args.profile_prefill:
+        del D
+        pb = synth.WORKLOADS["prefill"]
+        wlp = dataclasses.replace(pb, shape=dataclasses.replace(pb.shape, E=64))
+        T = args.profile_prefill
+        P = ds4moe.DeviceLayer(synth.make_layer(wlp), max_tokens=T)
+        x = torch.from_numpy(synth.activations(wlp, T)).cuda().view(torch.bfloat16)
+        for _ in range(2):
+            P.forward_grouped(x)
+        torch.cuda.synchronize()
+    assert ds4moe.last_device_error() == 0
+    print(json.dumps({"profile_case": "ok", "prefill_T": args.profile_prefill}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -373,7 +403,12 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--profile-case", action="store_true", help="small case for ncu captures (see profiles/)")
+    ap.add_argument("--profile-prefill", type=int, default=0, help="with --profile-case: also run a T-token prefill")
     args = ap.parse_args()
+    if args.profile_case:
+        run_profile_case(args)
+        return
     if args.impl == "reference":
         ws, rank = int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0"))
         run_reference(args, ws, rank)

@@ -35,12 +35,16 @@ struct ExpertsDev {
     Planes pd;  // planes of one down matrix [d x f]
 };
 
-constexpr int GU_THREADS = 384;
+constexpr int GU_THREADS = 256;
+constexpr int GU_PS = 2;  // shared-expert chunks in flight per warp
+constexpr int GU_PR = 4;  // routed row pairs in flight per warp
 constexpr int GU_TABLE_BYTES = 256 * 8 * 16;  // 8 lane-slots x 256 entries x 8 fp16
 
 // dynamic shared memory of the gate/up kernel: codebook table + fp32 copy of x
 __host__ __device__ constexpr int gu_smem_bytes(int d) { return GU_TABLE_BYTES + d * 4; }
-constexpr int DN_THREADS = 512;
+constexpr int DN_THREADS = 256;
+constexpr int DN_KB = 8;        // routed experts whose row loads are in flight together
+constexpr int DN_SH_MAX = 128;  // max shared-expert elements per lane (f_shared <= 4096)
 
 // Codebook table in shared memory: entry e, slot s (= lane & 7) at (e*8 + s)*16.
 __device__ __forceinline__ void build_codebook_table(const uint8_t *__restrict__ codebook, uint8_t *tbl) {
@@ -188,34 +192,45 @@ __global__ void __launch_bounds__(GU_THREADS, 1)
     }
     __syncthreads();
     const int n_sh = ex.fs > 0 ? ex.fs * NCH : 0;
-    const int n_items = n_sh + k * ex.f;
-    const int nw_total = gridDim.x * NWARP;
-    bool waited = false;
-    for (int it = blockIdx.x * NWARP + warp; it < n_items; it += nw_total) {
-        if (it < n_sh) {
-            // lane handles elements [c*CS + lane*EL, +EL) of the row; x comes from shared memory
-            const int r = it / NCH, c = it % NCH;
-            const size_t off = size_t(r) * d + size_t(c) * CS + size_t(lane) * EL;
-            uint4 gv[NCV], uv[NCV];
+    const int n_rt = k * ex.f;
+    const int gw = blockIdx.x * NWARP + warp, nw_total = gridDim.x * NWARP;
+
+    // Phase 1 (independent of the router, overlaps its tail under programmatic dependent launch):
+    // shared-expert row chunks, GU_PS per warp with all loads in flight before any math.
+    for (int base = gw * GU_PS; base < n_sh; base += nw_total * GU_PS) {
+        uint4 gv[GU_PS][NCV], uv[GU_PS][NCV];
 #pragma unroll
-            for (int v = 0; v < NCV; v++) {
-                gv[v] = ldg_nc_v4(ex.sh_gate + off + 8 * v);
-                uv[v] = ldg_nc_v4(ex.sh_up + off + 8 * v);
+        for (int p = 0; p < GU_PS; p++) {
+            const int it = base + p;
+            if (it < n_sh) {
+                const int r = it / NCH, c = it % NCH;
+                const size_t off = size_t(r) * d + size_t(c) * CS + size_t(lane) * EL;
+#pragma unroll
+                for (int v = 0; v < NCV; v++) {
+                    gv[p][v] = ldg_nc_v4(ex.sh_gate + off + 8 * v);
+                    uv[p][v] = ldg_nc_v4(ex.sh_up + off + 8 * v);
+                }
             }
+        }
+#pragma unroll
+        for (int p = 0; p < GU_PS; p++) {
+            const int it = base + p;
+            if (it >= n_sh) break;
+            const int r = it / NCH, c = it % NCH;
             float ag = 0.f, au = 0.f;
 #pragma unroll
             for (int v = 0; v < NCV; v++) {
                 const float4 xa = xsh[(c * (EL / 4) + 2 * v) * 32 + lane];
                 const float4 xb = xsh[(c * (EL / 4) + 2 * v + 1) * 32 + lane];
                 const float xf[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
-                const uint32_t gw[4] = {gv[v].x, gv[v].y, gv[v].z, gv[v].w};
-                const uint32_t uw[4] = {uv[v].x, uv[v].y, uv[v].z, uv[v].w};
+                const uint32_t gwv[4] = {gv[p][v].x, gv[p][v].y, gv[p][v].z, gv[p][v].w};
+                const uint32_t uwv[4] = {uv[p][v].x, uv[p][v].y, uv[p][v].z, uv[p][v].w};
 #pragma unroll
                 for (int i = 0; i < 4; i++) {
-                    ag = fmaf(bf16_lo(gw[i]), xf[2 * i], ag);
-                    ag = fmaf(bf16_hi(gw[i]), xf[2 * i + 1], ag);
-                    au = fmaf(bf16_lo(uw[i]), xf[2 * i], au);
-                    au = fmaf(bf16_hi(uw[i]), xf[2 * i + 1], au);
+                    ag = fmaf(bf16_lo(gwv[i]), xf[2 * i], ag);
+                    ag = fmaf(bf16_hi(gwv[i]), xf[2 * i + 1], ag);
+                    au = fmaf(bf16_lo(uwv[i]), xf[2 * i], au);
+                    au = fmaf(bf16_hi(uwv[i]), xf[2 * i + 1], au);
                 }
             }
             ag = warp_sum(ag);
@@ -224,28 +239,41 @@ __global__ void __launch_bounds__(GU_THREADS, 1)
                 sh_part[size_t(2 * c) * ex.fs + r] = ag;
                 sh_part[size_t(2 * c + 1) * ex.fs + r] = au;
             }
-        } else {
-            if (!waited) {
-                pdl_wait();
-                waited = true;
+        }
+    }
+
+    // Phase 2: routed experts' gate/up row pairs, GU_PR per warp with all loads in flight.
+    pdl_wait();
+    for (int base = gw * GU_PR; base < n_rt; base += nw_total * GU_PR) {
+        IqLane<VPL> Lg[GU_PR], Lu[GU_PR];
+        bool valid[GU_PR];
+#pragma unroll
+        for (int p = 0; p < GU_PR; p++) {
+            const int q = base + p;
+            valid[p] = false;
+            if (q < n_rt) {
+                const int j = q / ex.f, r = q % ex.f;
+                const int e = ids[j];
+                if (e >= 0 && e < ex.E) {
+                    valid[p] = true;
+                    iq_load<VPL>(Lg[p], ex.gate + size_t(e) * ex.gate_stride, ex.pg, r, d, lane);
+                    iq_load<VPL>(Lu[p], ex.up + size_t(e) * ex.up_stride, ex.pg, r, d, lane);
+                } else if (lane == 0) {
+                    set_device_error(DS4MOE_EDEVICE);
+                }
             }
-            const int q = it - n_sh;
-            const int j = q / ex.f, r = q % ex.f;
-            const int e = ids[j];
-            if (e < 0 || e >= ex.E) {
-                if (lane == 0) set_device_error(DS4MOE_EDEVICE);
-                continue;
-            }
-            IqLane<VPL> Lg, Lu;
-            iq_load<VPL>(Lg, ex.gate + size_t(e) * ex.gate_stride, ex.pg, r, d, lane);
-            iq_load<VPL>(Lu, ex.up + size_t(e) * ex.up_stride, ex.pg, r, d, lane);
-            float ag = iq_dot<VPL>(Lg, xh, tbl_lane, lane);
-            float au = iq_dot<VPL>(Lu, xh, tbl_lane, lane);
+        }
+#pragma unroll
+        for (int p = 0; p < GU_PR; p++) {
+            if (!valid[p]) continue;
+            const int q = base + p;
+            float ag = iq_dot<VPL>(Lg[p], xh, tbl_lane, lane);
+            float au = iq_dot<VPL>(Lu[p], xh, tbl_lane, lane);
             ag = warp_sum(ag);
             au = warp_sum(au);
             if (lane == 0) {
                 const float g = ag * inv_xs, u = au * inv_xs;
-                h_out[size_t(j) * ex.f + r] = silu(g) * u;
+                h_out[q] = silu(g) * u;  // q = j * f + r
             }
         }
     }
@@ -265,7 +293,7 @@ __host__ __device__ __forceinline__ DownSmem down_smem_layout(int k, int wpl, in
     s.hsl = s.hsum + k * wpl * 32 * 4;             // fs floats (lane-interleaved float4s)
     s.wsc = s.hsl + ((fs * 4 + 15) / 16) * 16;     // k floats
     s.eid = s.wsc + ((k * 4 + 15) / 16) * 16;      // k ints
-    s.total = s.eid + ((k * 4 + 15) / 16) * 16;
+    s.total = s.eid + ((2 * k * 4 + 15) / 16) * 16;  // eid[k] then the per-expert max[k]
     return s;
 }
 
@@ -289,47 +317,64 @@ __global__ void __launch_bounds__(DN_THREADS, 1)
     int *eid = reinterpret_cast<int *>(smem + L.eid);
 
     pdl_wait();
-    // stage routed h_j as scaled fp16 pairs (h[16s+p], h[16s+p+8]) in lane-interleaved order
-    for (int j = warp; j < k; j += NWARP) {
-        const float *hj = h + size_t(j) * f;
-        float mx = 0.f;
-        if (lane < active)
-            for (int i = 0; i < WPL; i++)
-                for (int e = 0; e < 16; e++) mx = fmaxf(mx, fabsf(hj[(lane * WPL + i) * 16 + e]));
-        mx = warp_max(mx);
-        const int he = pow2_exponent_for(mx, 6);
-        const float sc = ldexpf(1.f, he);
-        if (lane < active) {
-            for (int i = 0; i < WPL; i++) {
-                const float *src = hj + (lane * WPL + i) * 16;
-                __half2 pr[8];
-                float ssum = 0.f;
+    // stage routed h_j as scaled fp16 pairs (h[16s+p], h[16s+p+8]) in lane-interleaved order.
+    // pass 1: per-expert max |h| (non-negative floats order like their bit patterns)
+    int *hmax = reinterpret_cast<int *>(smem + L.eid) + k;  // k ints after eid[]
+    const int nsub = f / 16;                                 // 16-float sub-blocks per expert
+    for (int j = threadIdx.x; j < k; j += blockDim.x) hmax[j] = 0;
+    __syncthreads();
+    for (int q = threadIdx.x; q < k * nsub; q += blockDim.x) {
+        const float4 *src = reinterpret_cast<const float4 *>(h + size_t(q) * 16);
+        float m = 0.f;
 #pragma unroll
-                for (int p = 0; p < 8; p++) {
-                    pr[p] = __floats2half2_rn(src[p] * sc, src[p + 8] * sc);
-                    const float2 back = __half22float2(pr[p]);
-                    ssum += back.x + back.y;
-                }
-                hq[((j * WPL + i) * 2 + 0) * 32 + lane] = *reinterpret_cast<uint4 *>(&pr[0]);
-                hq[((j * WPL + i) * 2 + 1) * 32 + lane] = *reinterpret_cast<uint4 *>(&pr[4]);
-                hsum[(j * WPL + i) * 32 + lane] = ssum;
-            }
+        for (int i = 0; i < 4; i++) {
+            const float4 v = src[i];
+            m = fmaxf(m, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
         }
-        if (lane == 0) {
-            wsc[j] = wts[j] * ldexpf(1.f, -he);
-            eid[j] = ids[j];
-        }
+        atomicMax(&hmax[q / nsub], __float_as_int(m));
     }
     // shared expert: hs = silu(g) * u, element r at lane r/ESL, offset o = r%ESL -> float4 slot [o/4][lane]
     const int esl = fs / 32;
-    for (int r = threadIdx.x; r < fs; r += blockDim.x) {
-        float g = 0.f, u = 0.f;
+    for (int r4 = threadIdx.x * 4; r4 < fs; r4 += blockDim.x * 4) {
+        float4 g = make_float4(0.f, 0.f, 0.f, 0.f), u = g;
         for (int c = 0; c < nch; c++) {
-            g += sh_part[size_t(2 * c) * fs + r];
-            u += sh_part[size_t(2 * c + 1) * fs + r];
+            const float4 gc = *reinterpret_cast<const float4 *>(sh_part + size_t(2 * c) * fs + r4);
+            const float4 uc = *reinterpret_cast<const float4 *>(sh_part + size_t(2 * c + 1) * fs + r4);
+            g.x += gc.x; g.y += gc.y; g.z += gc.z; g.w += gc.w;
+            u.x += uc.x; u.y += uc.y; u.z += uc.z; u.w += uc.w;
         }
-        const int ln = r / esl, o = r % esl;
-        hsl[((o / 4) * 32 + ln) * 4 + (o % 4)] = silu(g) * u;
+        const int ln = r4 / esl, o = r4 % esl;
+        reinterpret_cast<float4 *>(hsl)[(o / 4) * 32 + ln] =
+            make_float4(silu(g.x) * u.x, silu(g.y) * u.y, silu(g.z) * u.z, silu(g.w) * u.w);
+    }
+    __syncthreads();
+    // pass 2: scale to fp16, pair, interleave; per-sub-block sums of the rounded values
+    for (int q = threadIdx.x; q < k * nsub; q += blockDim.x) {
+        const int j = q / nsub, sbk = q % nsub;
+        const int ln = sbk / WPL, i = sbk % WPL;
+        const float sc = ldexpf(1.f, pow2_exponent_for(__int_as_float(hmax[j]), 6));
+        const float4 *src = reinterpret_cast<const float4 *>(h + size_t(q) * 16);
+        float v[16];
+#pragma unroll
+        for (int t = 0; t < 4; t++) {
+            const float4 w = src[t];
+            v[4 * t] = w.x; v[4 * t + 1] = w.y; v[4 * t + 2] = w.z; v[4 * t + 3] = w.w;
+        }
+        __half2 pr[8];
+        float ssum = 0.f;
+#pragma unroll
+        for (int p = 0; p < 8; p++) {
+            pr[p] = __floats2half2_rn(v[p] * sc, v[p + 8] * sc);
+            const float2 back = __half22float2(pr[p]);
+            ssum += back.x + back.y;
+        }
+        hq[((j * WPL + i) * 2 + 0) * 32 + ln] = *reinterpret_cast<uint4 *>(&pr[0]);
+        hq[((j * WPL + i) * 2 + 1) * 32 + ln] = *reinterpret_cast<uint4 *>(&pr[4]);
+        hsum[(j * WPL + i) * 32 + ln] = ssum;
+    }
+    for (int j = threadIdx.x; j < k; j += blockDim.x) {
+        wsc[j] = wts[j] * ldexpf(1.f, -pow2_exponent_for(__int_as_float(hmax[j]), 6));
+        eid[j] = ids[j];
     }
     __syncthreads();
 
@@ -337,59 +382,75 @@ __global__ void __launch_bounds__(DN_THREADS, 1)
     const int n0 = blockIdx.x * rpc, n1 = min(d, n0 + rpc);
     const int nsbf = f / QK;
     const __half2 k1024 = __float2half2_rn(1024.f);
+    constexpr int SCW = (WPL + 3) / 4;
     for (int n = n0 + warp; n < n1; n += NWARP) {
         float acc = 0.f;
-        if (lane < active) {
-#pragma unroll 2
-            for (int j = 0; j < k; j++) {
-                const int e = eid[j];
-                if (e < 0 || e >= ex.E) {
-                    if (lane == 0) set_device_error(DS4MOE_EDEVICE);
-                    continue;
+        // shared-expert row: issue its loads first so they overlap the routed experts' math
+        uint4 shw[DN_SH_MAX / 8];
+        const __nv_bfloat16 *srow = ex.sh_down + size_t(n) * fs + size_t(lane) * esl;
+#pragma unroll
+        for (int i = 0; i < DN_SH_MAX / 8; i++)
+            if (i < esl / 8) shw[i] = ldg_nc_v4(srow + 8 * i);
+        for (int j0 = 0; j0 < k; j0 += DN_KB) {
+            uint32_t qw[DN_KB][WPL], scw[DN_KB][SCW], dmw[DN_KB];
+            bool ok[DN_KB];
+#pragma unroll
+            for (int jj = 0; jj < DN_KB; jj++) {
+                const int j = j0 + jj;
+                ok[jj] = false;
+                if (j < k && lane < active) {
+                    const int e = eid[j];
+                    if (e >= 0 && e < ex.E) {
+                        ok[jj] = true;
+                        const uint8_t *base = ex.down + size_t(e) * ex.down_stride;
+                        const uint8_t *qp = base + ex.pd.off[0] + size_t(n) * nsbf * 64 + lane * WPL * 4;
+                        const uint8_t *sp = base + ex.pd.off[1] + size_t(n) * nsbf * 16 + lane * WPL;
+                        dmw[jj] = ldg_nc_u32(base + ex.pd.off[2] + (size_t(n) * nsbf + (lane * WPL) / 16) * 4);
+                        if constexpr (WPL == 8) {
+                            const uint4 a = ldg_nc_v4(qp), b = ldg_nc_v4(qp + 16);
+                            qw[jj][0] = a.x; qw[jj][1] = a.y; qw[jj][2] = a.z; qw[jj][3] = a.w;
+                            qw[jj][4] = b.x; qw[jj][5] = b.y; qw[jj][6] = b.z; qw[jj][7] = b.w;
+                            const uint2 s2 = *reinterpret_cast<const uint2 *>(sp);
+                            scw[jj][0] = s2.x; scw[jj][1] = s2.y;
+                        } else if constexpr (WPL == 4) {
+                            const uint4 a = ldg_nc_v4(qp);
+                            qw[jj][0] = a.x; qw[jj][1] = a.y; qw[jj][2] = a.z; qw[jj][3] = a.w;
+                            scw[jj][0] = ldg_nc_u32(sp);
+                        } else if constexpr (WPL == 2) {
+                            const uint2 a = *reinterpret_cast<const uint2 *>(qp);
+                            qw[jj][0] = a.x; qw[jj][1] = a.y;
+                            scw[jj][0] = *reinterpret_cast<const uint16_t *>(sp);
+                        } else {
+                            qw[jj][0] = ldg_nc_u32(qp);
+                            scw[jj][0] = *sp;
+                        }
+                    } else if (lane == 0) {
+                        set_device_error(DS4MOE_EDEVICE);
+                    }
                 }
-                const uint8_t *base = ex.down + size_t(e) * ex.down_stride;
-                const uint8_t *qp = base + ex.pd.off[0] + size_t(n) * nsbf * 64 + lane * WPL * 4;
-                const uint8_t *sp = base + ex.pd.off[1] + size_t(n) * nsbf * 16 + lane * WPL;
-                const uint32_t dm =
-                    ldg_nc_u32(base + ex.pd.off[2] + (size_t(n) * nsbf + (lane * WPL) / 16) * 4);
-                uint32_t qw[WPL];
-                uint32_t scw[(WPL + 3) / 4];
-                if constexpr (WPL == 8) {
-                    uint4 a = ldg_nc_v4(qp), b = ldg_nc_v4(qp + 16);
-                    qw[0] = a.x; qw[1] = a.y; qw[2] = a.z; qw[3] = a.w;
-                    qw[4] = b.x; qw[5] = b.y; qw[6] = b.z; qw[7] = b.w;
-                    uint2 s2 = *reinterpret_cast<const uint2 *>(sp);
-                    scw[0] = s2.x; scw[1] = s2.y;
-                } else if constexpr (WPL == 4) {
-                    uint4 a = ldg_nc_v4(qp);
-                    qw[0] = a.x; qw[1] = a.y; qw[2] = a.z; qw[3] = a.w;
-                    scw[0] = ldg_nc_u32(sp);
-                } else if constexpr (WPL == 2) {
-                    uint2 a = *reinterpret_cast<const uint2 *>(qp);
-                    qw[0] = a.x; qw[1] = a.y;
-                    scw[0] = *reinterpret_cast<const uint16_t *>(sp);
-                } else {
-                    qw[0] = ldg_nc_u32(qp);
-                    scw[0] = *sp;
-                }
-                const float dd = half_bits_to_float(uint16_t(dm & 0xFFFF));
-                const float dmin = half_bits_to_float(uint16_t(dm >> 16));
+            }
+#pragma unroll
+            for (int jj = 0; jj < DN_KB; jj++) {
+                if (!ok[jj]) continue;
+                const int j = j0 + jj;
+                const float dd = half_bits_to_float(uint16_t(dmw[jj] & 0xFFFF));
+                const float dmin = half_bits_to_float(uint16_t(dmw[jj] >> 16));
                 float part = 0.f;
 #pragma unroll
                 for (int i = 0; i < WPL; i++) {
                     const uint4 hA = hq[((j * WPL + i) * 2 + 0) * 32 + lane];
                     const uint4 hB = hq[((j * WPL + i) * 2 + 1) * 32 + lane];
                     const uint32_t hp[8] = {hA.x, hA.y, hA.z, hA.w, hB.x, hB.y, hB.z, hB.w};
-                    __half2 a = __float2half2_rn(0.f), b = __float2half2_rn(0.f);
+                    __half2 a2 = __float2half2_rn(0.f), b2 = __float2half2_rn(0.f);
 #pragma unroll
                     for (int p = 0; p < 8; p++) {
-                        const uint32_t v = ((qw[i] >> (2 * p)) & 0x00030003u) | 0x64006400u;
+                        const uint32_t v = ((qw[jj][i] >> (2 * p)) & 0x00030003u) | 0x64006400u;
                         const __half2 q2 = __hsub2(u32_as_half2(v), k1024);
-                        if (p & 1) b = __hfma2(q2, u32_as_half2(hp[p]), b);
-                        else a = __hfma2(q2, u32_as_half2(hp[p]), a);
+                        if (p & 1) b2 = __hfma2(q2, u32_as_half2(hp[p]), b2);
+                        else a2 = __hfma2(q2, u32_as_half2(hp[p]), a2);
                     }
-                    const float2 fa = __half22float2(a), fb = __half22float2(b);
-                    const uint32_t scb = (scw[i / 4] >> (8 * (i % 4))) & 0xFFu;
+                    const float2 fa = __half22float2(a2), fb = __half22float2(b2);
+                    const uint32_t scb = (scw[jj][i / 4] >> (8 * (i % 4))) & 0xFFu;
                     const float sc = float(scb & 15u), mn = float(scb >> 4);
                     part += (dd * sc) * ((fa.x + fa.y) + (fb.x + fb.y)) - (dmin * mn) * hsum[(j * WPL + i) * 32 + lane];
                 }
@@ -397,10 +458,11 @@ __global__ void __launch_bounds__(DN_THREADS, 1)
             }
         }
         if (fs > 0) {
-            const __nv_bfloat16 *row = ex.sh_down + size_t(n) * fs + size_t(lane) * esl;
             const float4 *h4 = reinterpret_cast<const float4 *>(hsl);
-            for (int i = 0; i < esl / 8; i++) {
-                const uint4 wv = ldg_nc_v4(row + 8 * i);
+#pragma unroll
+            for (int i = 0; i < DN_SH_MAX / 8; i++) {
+                if (i >= esl / 8) break;
+                const uint4 wv = shw[i];
                 const float4 ha = h4[(2 * i) * 32 + lane], hb = h4[(2 * i + 1) * 32 + lane];
                 acc = fmaf(bf16_lo(wv.x), ha.x, acc);
                 acc = fmaf(bf16_hi(wv.x), ha.y, acc);

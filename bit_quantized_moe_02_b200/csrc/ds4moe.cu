@@ -2,10 +2,12 @@
 // kernel launches.  One translation unit: the kernels live in the headers
 // included below.
 #include <stdio.h>
+#include <stdlib.h>
 
 #include "common.cuh"
 #include "decode.cuh"
 #include "grouped_mma.cuh"
+#include "grouped_tc.cuh"
 #include "permute.cuh"
 #include "prepare.cuh"
 #include "route.cuh"
@@ -129,11 +131,23 @@ struct GroupedWs {
     uint64_t total_grouped, total_decode;
     int nblk, max_tiles;
 };
+// The tcgen05 kernels run the grouped GEMMs; DS4MOE_GROUPED=mma selects the warp-level mma.sync kernels
+// instead (same results within rounding; kept for A/B measurement).
+bool use_tc_grouped() {
+    static int v = -1;
+    if (v < 0) {
+        const char *e = getenv("DS4MOE_GROUPED");
+        v = (e && e[0] == 'm') ? 0 : 1;
+    }
+    return v == 1;
+}
+int grouped_tile_n() { return use_tc_grouped() ? tc::NT : TILE_N; }
+
 GroupedWs grouped_ws(const ds4moe_experts *ex, int T, int k) {
     GroupedWs w;
     const uint64_t N = uint64_t(T) * k;
     w.nblk = int((N + PERM_BLOCK - 1) / PERM_BLOCK);
-    w.max_tiles = int(ex->E + (N + TILE_N - 1) / TILE_N);
+    w.max_tiles = int(ex->E + (N + 63) / 64);  // enough for 64- and 128-token tiles
     uint64_t o = 0;
     auto take = [&](uint64_t bytes) {
         uint64_t r = o;
@@ -163,12 +177,20 @@ GroupedWs grouped_ws(const ds4moe_experts *ex, int T, int k) {
 
 // ---- grouped launch sequence --------------------------------------------------------------------------
 
+// row_units: rows of one A matrix (f for gate/up, d for down); col_tiles: token tiles (upper bound)
 template <int AFMT, bool GATEUP>
-ds4moe_status launch_grouped(const GroupedArgs &ga, int row_tiles, int col_tiles, cudaStream_t st) {
-    auto kern = grouped_mma_kernel<AFMT, GATEUP>;
-    if (!set_smem(kern, GM_SMEM)) return DS4MOE_ECUDA;
-    if (row_tiles <= 0 || col_tiles <= 0) return DS4MOE_OK;
-    kern<<<dim3(row_tiles, col_tiles), GM_THREADS, GM_SMEM, st>>>(ga);
+ds4moe_status launch_grouped(const GroupedArgs &ga, int row_units, int col_tiles, cudaStream_t st) {
+    if (row_units <= 0 || col_tiles <= 0) return DS4MOE_OK;
+    if (use_tc_grouped()) {
+        auto kern = tc::grouped_tc_kernel<AFMT, GATEUP>;
+        constexpr int smem = tc::Cfg<GATEUP>::SMEM;
+        if (!set_smem(kern, smem)) return DS4MOE_ECUDA;
+        kern<<<dim3(row_units / tc::M, col_tiles), tc::THREADS, smem, st>>>(ga);
+    } else {
+        auto kern = grouped_mma_kernel<AFMT, GATEUP>;
+        if (!set_smem(kern, GM_SMEM)) return DS4MOE_ECUDA;
+        kern<<<dim3(GATEUP ? row_units / 64 : row_units / GM_M, col_tiles), GM_THREADS, GM_SMEM, st>>>(ga);
+    }
     DS4_CHECK_LAUNCH();
     return DS4MOE_OK;
 }
@@ -198,7 +220,9 @@ ds4moe_status run_grouped(const ds4moe_experts *ex, const void *x, int T, const 
     const size_t hist_smem = size_t(ex->E) * 4;
     perm_count_kernel<<<W.nblk, PERM_BLOCK, hist_smem, st>>>(ids, N, ex->E, blk);
     DS4_CHECK_LAUNCH();
-    perm_scan_kernel<<<1, 1024, 0, st>>>(blk, W.nblk, ex->E, counts, offsets, tile_e, tile_pos0, tile_cnt, meta);
+    const int tile_n = grouped_tile_n();
+    perm_scan_kernel<<<1, 1024, 0, st>>>(blk, W.nblk, ex->E, tile_n, counts, offsets, tile_e, tile_pos0, tile_cnt,
+                                         meta);
     DS4_CHECK_LAUNCH();
     perm_scatter_kernel<<<W.nblk, PERM_BLOCK, hist_smem, st>>>(ids, weights, N, k, ex->E, blk, perm_tok, perm_w,
                                                                inv_perm);
@@ -212,8 +236,8 @@ ds4moe_status run_grouped(const ds4moe_experts *ex, const void *x, int T, const 
     g1.tile_e = tile_e; g1.tile_pos0 = tile_pos0; g1.tile_cnt = tile_cnt; g1.n_tiles = meta;
     g1.out = h16; g1.ldo = ex->f;
     ds4moe_status s;
-    if (ex->fmt_gate == DS4MOE_FMT_IQ2X) s = launch_grouped<DS4MOE_FMT_IQ2X, true>(g1, ex->f / 64, W.max_tiles, st);
-    else s = launch_grouped<DS4MOE_FMT_Q4K, true>(g1, ex->f / 64, W.max_tiles, st);
+    if (ex->fmt_gate == DS4MOE_FMT_IQ2X) s = launch_grouped<DS4MOE_FMT_IQ2X, true>(g1, ex->f, W.max_tiles, st);
+    else s = launch_grouped<DS4MOE_FMT_Q4K, true>(g1, ex->f, W.max_tiles, st);
     if (s != DS4MOE_OK) return s;
 
     // routed GEMM-2: down -> y_perm (scaled by the routing weight)
@@ -222,22 +246,22 @@ ds4moe_status run_grouped(const ds4moe_experts *ex, const void *x, int T, const 
     g2.b_src = h16; g2.b_rowidx = nullptr; g2.b_colscale = nullptr;
     g2.tile_e = tile_e; g2.tile_pos0 = tile_pos0; g2.tile_cnt = tile_cnt; g2.n_tiles = meta;
     g2.pos_weight = perm_w; g2.out = y_perm; g2.ldo = ex->d;
-    if (ex->fmt_down == DS4MOE_FMT_Q2K) s = launch_grouped<DS4MOE_FMT_Q2K, false>(g2, ex->d / GM_M, W.max_tiles, st);
-    else s = launch_grouped<DS4MOE_FMT_Q4K, false>(g2, ex->d / GM_M, W.max_tiles, st);
+    if (ex->fmt_down == DS4MOE_FMT_Q2K) s = launch_grouped<DS4MOE_FMT_Q2K, false>(g2, ex->d, W.max_tiles, st);
+    else s = launch_grouped<DS4MOE_FMT_Q4K, false>(g2, ex->d, W.max_tiles, st);
     if (s != DS4MOE_OK) return s;
 
     if (ex->f_shared > 0) {
-        const int ct = (T + GM_N - 1) / GM_N;
+        const int ct = (T + tile_n - 1) / tile_n;
         GroupedArgs s1 = {};
         s1.a0 = static_cast<const uint8_t *>(ex->sh_gate); s1.a1 = static_cast<const uint8_t *>(ex->sh_up);
         s1.a_stride = 0; s1.rows = ex->f_shared; s1.K = ex->d;
         s1.b_src = x16; s1.b_colscale = xinv; s1.n_pos = T; s1.out = hs; s1.ldo = ex->f_shared;
-        s = launch_grouped<DS4MOE_FMT_BF16, true>(s1, ex->f_shared / 64, ct, st);
+        s = launch_grouped<DS4MOE_FMT_BF16, true>(s1, ex->f_shared, ct, st);
         if (s != DS4MOE_OK) return s;
         GroupedArgs s2 = {};
         s2.a0 = static_cast<const uint8_t *>(ex->sh_down); s2.a_stride = 0; s2.rows = ex->d; s2.K = ex->f_shared;
         s2.b_src = hs; s2.n_pos = T; s2.out = y_shared; s2.ldo = ex->d;
-        s = launch_grouped<DS4MOE_FMT_BF16, false>(s2, ex->d / GM_M, ct, st);
+        s = launch_grouped<DS4MOE_FMT_BF16, false>(s2, ex->d, ct, st);
         if (s != DS4MOE_OK) return s;
     }
     return DS4MOE_OK;

@@ -319,7 +319,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_tc_kernel(GroupedArgs a) {
         if (warp < W_A0 + 4) {
             const int q = warp - W_A0;  // TMEM lane quarter
             const int r = q * 32 + lane;
-            const bool ok = mbar_wait(accum_bar, 0, abort_flag) && !*abort_flag;
+            const bool ok = __all_sync(0xffffffffu, mbar_wait(accum_bar, 0, abort_flag) && !*abort_flag);
             tc_fence_after();
             if (ok) {
                 const uint32_t tq = tmem + (uint32_t(q * 32) << 16);

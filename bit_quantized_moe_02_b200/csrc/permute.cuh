@@ -13,7 +13,7 @@
 namespace ds4 {
 
 constexpr int PERM_BLOCK = 1024;
-constexpr int TILE_N = 64;  // tokens per grouped-GEMM tile
+constexpr int TILE_N = 64;  // tokens per tile of the mma.sync grouped kernel
 
 // x16[t] = fp16(x[t] * 2^e_t) with max|x16[t]| in [2^13, 2^14); xinv[t] = 2^-e_t.
 __global__ void __launch_bounds__(256) prep_x_kernel(const __nv_bfloat16 *__restrict__ x, int d,
@@ -65,7 +65,7 @@ __global__ void __launch_bounds__(PERM_BLOCK) perm_count_kernel(const int32_t *_
 
 // Single CTA: expert offsets, per-block scatter bases, and the token-tile list.
 // meta = {n_tiles, n_used_experts}; counts/offsets [E].
-__global__ void __launch_bounds__(1024) perm_scan_kernel(int32_t *__restrict__ blk_counts, int nblk, int E,
+__global__ void __launch_bounds__(1024) perm_scan_kernel(int32_t *__restrict__ blk_counts, int nblk, int E, int tile_n,
                                                          int32_t *__restrict__ counts, int32_t *__restrict__ offsets,
                                                          int32_t *__restrict__ tile_e, int32_t *__restrict__ tile_pos0,
                                                          int32_t *__restrict__ tile_cnt, int32_t *__restrict__ meta) {
@@ -75,7 +75,7 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(int32_t *__restrict__ b
     int tot = 0;
     if (e < E)
         for (int b = 0; b < nblk; b++) tot += blk_counts[size_t(b) * E + e];
-    const int nt = (tot + TILE_N - 1) / TILE_N;
+    const int nt = (tot + tile_n - 1) / tile_n;
     s_tot[e] = e < E ? tot : 0;
     s_nt[e] = e < E ? nt : 0;
     __syncthreads();
@@ -104,8 +104,8 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(int32_t *__restrict__ b
         }
         for (int i = 0; i < nt; i++) {
             tile_e[toff + i] = e;
-            tile_pos0[toff + i] = off + i * TILE_N;
-            tile_cnt[toff + i] = min(TILE_N, tot - i * TILE_N);
+            tile_pos0[toff + i] = off + i * tile_n;
+            tile_cnt[toff + i] = min(tile_n, tot - i * tile_n);
         }
     }
     if (e == 1023) {
