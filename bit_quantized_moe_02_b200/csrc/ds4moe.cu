@@ -1,11 +1,13 @@
 // ds4moe C ABI (include/ds4moe.h): argument checks, workspace carving and
 // kernel launches.  One translation unit: the kernels live in the headers
 // included below.
+#include <cudaTypedefs.h>
 #include <stdio.h>
 #include <stdlib.h>
 
 #include "common.cuh"
 #include "decode.cuh"
+#include "decode_ring.cuh"
 #include "grouped_mma.cuh"
 #include "grouped_tc.cuh"
 #include "permute.cuh"
@@ -58,6 +60,37 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
+// ---- TMA tensor maps ----------------------------------------------------------------------------------------
+//
+// The tcgen05 kernels load their token operand (a row-major fp16 matrix, rows x cols) with 2D tensor copies:
+// box = 64 columns (128 bytes, the swizzle span) x 128 rows, 128-byte swizzle, zero fill past the last row.
+// The encoder comes from the driver through the runtime's entry-point query (no link against libcuda).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+        tried = true;
+    }
+    return fn;
+}
+
+bool make_token_map(CUtensorMap *m, const __half *base, uint64_t rows, uint64_t cols) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc || !base || rows == 0 || cols % 64 || !aligned16(base)) return false;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * 2};
+    const cuuint32_t box[2] = {uint32_t(tc::BK), uint32_t(tc::NT)};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<__half *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 bool fmt_quant(int f) { return f == DS4MOE_FMT_IQ2X || f == DS4MOE_FMT_Q2K || f == DS4MOE_FMT_Q4K; }
@@ -114,11 +147,27 @@ struct DecodeWs {
     uint64_t h, sh_part, total;
     int nch;
 };
+// The ring-pipelined decode kernels cover d in {2048, 4096} (gate/up) and f = 2048 with f_shared a multiple of
+// 512 (down); other shapes run the register-batched kernels.
+// DS4MOE_DECODE=regs selects the register-batched kernels everywhere (A/B measurement).
+bool decode_regs_forced() {
+    static int v = -1;
+    if (v < 0) {
+        const char *e = getenv("DS4MOE_DECODE");
+        v = (e && e[0] == 'r' && e[1] == 'e') ? 1 : 0;
+    }
+    return v == 1;
+}
+bool gateup_ring(const ds4moe_experts *ex) { return !decode_regs_forced() && (ex->d == 4096 || ex->d == 2048); }
+bool down_ring(const ds4moe_experts *ex) {
+    return !decode_regs_forced() && ex->f == 2048 && ex->f_shared % 512 == 0 && ex->d <= 8192;
+}
+
 DecodeWs decode_ws(const ds4moe_experts *ex, int k) {
     DecodeWs w;
     const int vpl = ex->d / QK;
     const int ncv = vpl < 4 ? vpl : 4;
-    w.nch = vpl / ncv;
+    w.nch = gateup_ring(ex) ? ex->d / 512 : vpl / ncv;  // shared-expert partial-sum chunks per row
     w.h = 0;
     w.sh_part = a256(uint64_t(k) * ex->f * 4);
     w.total = w.sh_part + a256(uint64_t(w.nch) * 2 * (ex->f_shared > 0 ? ex->f_shared : 1) * 4);
@@ -126,7 +175,7 @@ DecodeWs decode_ws(const ds4moe_experts *ex, int k) {
 }
 
 struct GroupedWs {
-    uint64_t x16, xinv, blk, counts, offsets, tile_e, tile_pos0, tile_cnt, meta, perm_tok, perm_w, h16, hs;
+    uint64_t x16, xinv, blk, counts, offsets, tile_e, tile_pos0, tile_cnt, meta, perm_tok, perm_w, x_perm, h16, hs;
     uint64_t y_perm, inv, y_shared;  // only used when decode B > 1 runs through the grouped path
     uint64_t total_grouped, total_decode;
     int nblk, max_tiles;
@@ -165,6 +214,7 @@ GroupedWs grouped_ws(const ds4moe_experts *ex, int T, int k) {
     w.meta = take(16);
     w.perm_tok = take(N * 4);
     w.perm_w = take(N * 4);
+    w.x_perm = take(use_tc_grouped() ? N * ex->d * 2 : 0);
     w.h16 = take(N * ex->f * 2);
     w.hs = take(uint64_t(T) * (ex->f_shared > 0 ? ex->f_shared : 1) * 2);
     w.total_grouped = o;
@@ -177,15 +227,19 @@ GroupedWs grouped_ws(const ds4moe_experts *ex, int T, int k) {
 
 // ---- grouped launch sequence --------------------------------------------------------------------------
 
-// row_units: rows of one A matrix (f for gate/up, d for down); col_tiles: token tiles (upper bound)
+// row_units: rows of one A matrix (f for gate/up, d for down); col_tiles: token tiles (upper bound).
+// b_tma / b_rows: the token operand as the tcgen05 kernel reads it (row-major fp16, b_rows x ga.K).
 template <int AFMT, bool GATEUP>
-ds4moe_status launch_grouped(const GroupedArgs &ga, int row_units, int col_tiles, cudaStream_t st) {
+ds4moe_status launch_grouped(const GroupedArgs &ga, int row_units, int col_tiles, const __half *b_tma,
+                             uint64_t b_rows, cudaStream_t st) {
     if (row_units <= 0 || col_tiles <= 0) return DS4MOE_OK;
     if (use_tc_grouped()) {
+        CUtensorMap tmap;
+        if (!make_token_map(&tmap, b_tma, b_rows, uint64_t(ga.K))) return DS4MOE_ECUDA;
         auto kern = tc::grouped_tc_kernel<AFMT, GATEUP>;
         constexpr int smem = tc::Cfg<GATEUP>::SMEM;
         if (!set_smem(kern, smem)) return DS4MOE_ECUDA;
-        kern<<<dim3(row_units / tc::M, col_tiles), tc::THREADS, smem, st>>>(ga);
+        kern<<<dim3(row_units / tc::M, col_tiles), tc::THREADS, smem, st>>>(ga, tmap);
     } else {
         auto kern = grouped_mma_kernel<AFMT, GATEUP>;
         if (!set_smem(kern, GM_SMEM)) return DS4MOE_ECUDA;
@@ -211,6 +265,7 @@ ds4moe_status run_grouped(const ds4moe_experts *ex, const void *x, int T, const 
     int32_t *meta = reinterpret_cast<int32_t *>(ws + W.meta);
     int32_t *perm_tok = reinterpret_cast<int32_t *>(ws + W.perm_tok);
     float *perm_w = reinterpret_cast<float *>(ws + W.perm_w);
+    __half *x_perm = reinterpret_cast<__half *>(ws + W.x_perm);
     __half *h16 = reinterpret_cast<__half *>(ws + W.h16);
     __half *hs = reinterpret_cast<__half *>(ws + W.hs);
     const __nv_bfloat16 *xb = static_cast<const __nv_bfloat16 *>(x);
@@ -227,6 +282,10 @@ ds4moe_status run_grouped(const ds4moe_experts *ex, const void *x, int T, const 
     perm_scatter_kernel<<<W.nblk, PERM_BLOCK, hist_smem, st>>>(ids, weights, N, k, ex->E, blk, perm_tok, perm_w,
                                                                inv_perm);
     DS4_CHECK_LAUNCH();
+    if (use_tc_grouped()) {
+        gather_rows_kernel<<<(N + 7) / 8, 256, 0, st>>>(x16, ex->d, perm_tok, N, x_perm);
+        DS4_CHECK_LAUNCH();
+    }
 
     // routed GEMM-1: gate/up -> h16
     GroupedArgs g1 = {};
@@ -236,8 +295,8 @@ ds4moe_status run_grouped(const ds4moe_experts *ex, const void *x, int T, const 
     g1.tile_e = tile_e; g1.tile_pos0 = tile_pos0; g1.tile_cnt = tile_cnt; g1.n_tiles = meta;
     g1.out = h16; g1.ldo = ex->f;
     ds4moe_status s;
-    if (ex->fmt_gate == DS4MOE_FMT_IQ2X) s = launch_grouped<DS4MOE_FMT_IQ2X, true>(g1, ex->f, W.max_tiles, st);
-    else s = launch_grouped<DS4MOE_FMT_Q4K, true>(g1, ex->f, W.max_tiles, st);
+    if (ex->fmt_gate == DS4MOE_FMT_IQ2X) s = launch_grouped<DS4MOE_FMT_IQ2X, true>(g1, ex->f, W.max_tiles, x_perm, N, st);
+    else s = launch_grouped<DS4MOE_FMT_Q4K, true>(g1, ex->f, W.max_tiles, x_perm, N, st);
     if (s != DS4MOE_OK) return s;
 
     // routed GEMM-2: down -> y_perm (scaled by the routing weight)
@@ -246,8 +305,8 @@ ds4moe_status run_grouped(const ds4moe_experts *ex, const void *x, int T, const 
     g2.b_src = h16; g2.b_rowidx = nullptr; g2.b_colscale = nullptr;
     g2.tile_e = tile_e; g2.tile_pos0 = tile_pos0; g2.tile_cnt = tile_cnt; g2.n_tiles = meta;
     g2.pos_weight = perm_w; g2.out = y_perm; g2.ldo = ex->d;
-    if (ex->fmt_down == DS4MOE_FMT_Q2K) s = launch_grouped<DS4MOE_FMT_Q2K, false>(g2, ex->d, W.max_tiles, st);
-    else s = launch_grouped<DS4MOE_FMT_Q4K, false>(g2, ex->d, W.max_tiles, st);
+    if (ex->fmt_down == DS4MOE_FMT_Q2K) s = launch_grouped<DS4MOE_FMT_Q2K, false>(g2, ex->d, W.max_tiles, h16, N, st);
+    else s = launch_grouped<DS4MOE_FMT_Q4K, false>(g2, ex->d, W.max_tiles, h16, N, st);
     if (s != DS4MOE_OK) return s;
 
     if (ex->f_shared > 0) {
@@ -256,12 +315,12 @@ ds4moe_status run_grouped(const ds4moe_experts *ex, const void *x, int T, const 
         s1.a0 = static_cast<const uint8_t *>(ex->sh_gate); s1.a1 = static_cast<const uint8_t *>(ex->sh_up);
         s1.a_stride = 0; s1.rows = ex->f_shared; s1.K = ex->d;
         s1.b_src = x16; s1.b_colscale = xinv; s1.n_pos = T; s1.out = hs; s1.ldo = ex->f_shared;
-        s = launch_grouped<DS4MOE_FMT_BF16, true>(s1, ex->f_shared, ct, st);
+        s = launch_grouped<DS4MOE_FMT_BF16, true>(s1, ex->f_shared, ct, x16, T, st);
         if (s != DS4MOE_OK) return s;
         GroupedArgs s2 = {};
         s2.a0 = static_cast<const uint8_t *>(ex->sh_down); s2.a_stride = 0; s2.rows = ex->d; s2.K = ex->f_shared;
         s2.b_src = hs; s2.n_pos = T; s2.out = y_shared; s2.ldo = ex->d;
-        s = launch_grouped<DS4MOE_FMT_BF16, false>(s2, ex->d, ct, st);
+        s = launch_grouped<DS4MOE_FMT_BF16, false>(s2, ex->d, ct, hs, T, st);
         if (s != DS4MOE_OK) return s;
     }
     return DS4MOE_OK;
@@ -362,10 +421,16 @@ ds4moe_status ds4moe_dequant(ds4moe_fmt fmt, const void *prepared, const uint8_t
     return DS4MOE_OK;
 }
 
+// Router workspace: logits [T x E] fp32; for the tensor-core path (T > ROUTE_SMALL_T, E a multiple of 128)
+// also the per-token scaled fp16 copy of x and its scales.
+static bool route_tc(int T, int d, int E) { return T > ROUTE_SMALL_T && E % tc::M == 0 && d % QK == 0; }
+
 size_t ds4moe_route_workspace_size(int T, int d, int E) {
-    (void)d;
-    if (T < 0 || E <= 0) return 0;
-    return a256(uint64_t(T > 0 ? T : 1) * E * 4);
+    if (T < 0 || E <= 0 || d <= 0) return 0;
+    const uint64_t TT = T > 0 ? T : 1;
+    uint64_t n = a256(TT * E * 4);
+    if (route_tc(T, d, E)) n += a256(TT * d * 2) + a256(TT * 4);
+    return n;
 }
 
 ds4moe_status ds4moe_route(const void *x_bf16, int T, int d, const void *w_router_f16, const float *bias, int E,
@@ -374,19 +439,46 @@ ds4moe_status ds4moe_route(const void *x_bf16, int T, int d, const void *w_route
     if (T < 0 || d <= 0 || d % QK || E <= 0 || E > 1024 || k < 1 || k > E || k > 32) return DS4MOE_EINVAL;
     if (T == 0) return DS4MOE_OK;
     if (!x_bf16 || !w_router_f16 || !ids || !weights || !ws) return DS4MOE_EINVAL;
-    if (!aligned16(x_bf16) || !aligned16(w_router_f16)) return DS4MOE_EINVAL;
+    if (!aligned16(x_bf16) || !aligned16(w_router_f16) || !aligned256(ws)) return DS4MOE_EINVAL;
     if (ws_bytes < ds4moe_route_workspace_size(T, d, E)) return DS4MOE_ENOWORKSPACE;
     float *logits = static_cast<float *>(ws);
     const __nv_bfloat16 *x = static_cast<const __nv_bfloat16 *>(x_bf16);
     const __half *wr = static_cast<const __half *>(w_router_f16);
+    cudaStream_t st = cs(stream);
+    const float *late_bias = nullptr;
     if (T <= ROUTE_SMALL_T) {
-        route_logits_small_kernel<<<(E + 1) / 2, 256, 0, cs(stream)>>>(x, T, d, wr, bias, E, logits);
+        route_logits_small_kernel<<<(E + 1) / 2, 256, 0, st>>>(x, T, d, wr, bias, E, logits);
+    } else if (route_tc(T, d, E)) {
+        // fp16 x fp16 products are exact on the tensor cores (W_r is fp16; x is scaled per token by a power of
+        // two into fp16 range), accumulation in fp32: logits[t][e] = (W_r x16[t])[e] * 2^-e_t
+        uint8_t *w8 = static_cast<uint8_t *>(ws);
+        __half *x16 = reinterpret_cast<__half *>(w8 + a256(uint64_t(T) * E * 4));
+        float *xinv = reinterpret_cast<float *>(w8 + a256(uint64_t(T) * E * 4) + a256(uint64_t(T) * d * 2));
+        prep_x_kernel<<<T, 256, 0, st>>>(x, d, x16, xinv);
+        DS4_CHECK_LAUNCH();
+        GroupedArgs g = {};
+        g.a0 = static_cast<const uint8_t *>(w_router_f16);
+        g.a_stride = 0; g.rows = E; g.K = d;
+        g.b_src = x16; g.b_colscale = xinv; g.n_pos = T;
+        g.out = logits; g.ldo = E;
+        CUtensorMap tmap;
+        if (!make_token_map(&tmap, x16, uint64_t(T), uint64_t(d))) return DS4MOE_ECUDA;
+        auto kern = tc::grouped_tc_kernel<tc::FMT_F16, false>;
+        constexpr int smem = tc::Cfg<false>::SMEM;
+        if (!set_smem(kern, smem)) return DS4MOE_ECUDA;
+        kern<<<dim3(E / tc::M, (T + tc::NT - 1) / tc::NT), tc::THREADS, smem, st>>>(g, tmap);
+        late_bias = bias;
     } else {
-        route_logits_tiled_kernel<<<dim3((T + 63) / 64, (E + 63) / 64), 256, 0, cs(stream)>>>(x, T, d, wr, bias, E,
-                                                                                             logits);
+        route_logits_tiled_kernel<<<dim3((T + 63) / 64, (E + 63) / 64), 256, 0, st>>>(x, T, d, wr, bias, E, logits);
     }
     DS4_CHECK_LAUNCH();
-    route_topk_kernel<<<(T + 7) / 8, 256, 0, cs(stream)>>>(logits, T, E, k, ids, weights);
+    const unsigned tg = unsigned((T + 7) / 8);
+    if (E <= 32) route_topk_kernel<1><<<tg, 256, 0, st>>>(logits, T, E, k, late_bias, ids, weights);
+    else if (E <= 64) route_topk_kernel<2><<<tg, 256, 0, st>>>(logits, T, E, k, late_bias, ids, weights);
+    else if (E <= 128) route_topk_kernel<4><<<tg, 256, 0, st>>>(logits, T, E, k, late_bias, ids, weights);
+    else if (E <= 256) route_topk_kernel<8><<<tg, 256, 0, st>>>(logits, T, E, k, late_bias, ids, weights);
+    else if (E <= 512) route_topk_kernel<16><<<tg, 256, 0, st>>>(logits, T, E, k, late_bias, ids, weights);
+    else route_topk_kernel<32><<<tg, 256, 0, st>>>(logits, T, E, k, late_bias, ids, weights);
     DS4_CHECK_LAUNCH();
     return DS4MOE_OK;
 }
@@ -448,6 +540,22 @@ ds4moe_status ds4moe_decode_gateup(const ds4moe_experts *ex, const void *x_bf16,
     const int grid = num_sms();
     cudaStream_t st = cs(stream);
     cudaError_t err;
+    if (gateup_ring(ex)) {
+        if (ex->d == 4096) {
+            if (!set_smem(decode_gateup_ring_kernel<16>, GR_DYN)) return DS4MOE_ECUDA;
+            err = launch_pdl(decode_gateup_ring_kernel<16>, dim3(grid), dim3(GR_THREADS), size_t(GR_DYN), st, D, x, ids,
+                             k, h, shp);
+        } else {
+            if (!set_smem(decode_gateup_ring_kernel<8>, GR_DYN)) return DS4MOE_ECUDA;
+            err = launch_pdl(decode_gateup_ring_kernel<8>, dim3(grid), dim3(GR_THREADS), size_t(GR_DYN), st, D, x, ids,
+                             k, h, shp);
+        }
+        if (err != cudaSuccess) {
+            (void)cudaGetLastError();
+            return DS4MOE_ECUDA;
+        }
+        return DS4MOE_OK;
+    }
     switch (ex->d / QK) {
 #define GU_CASE(V)                                                                                              \
     case V:                                                                                                     \
@@ -485,6 +593,17 @@ ds4moe_status ds4moe_decode_down(const ds4moe_experts *ex, const int32_t *ids, c
     const DownSmem L = down_smem_layout(k, wpl, ex->f_shared);
     cudaStream_t st = cs(stream);
     cudaError_t err;
+    if (down_ring(ex)) {
+        const DownRingSmem RL = down_ring_layout(k, ex->f_shared);
+        if (!set_smem(decode_down_ring_kernel, RL.total)) return DS4MOE_ECUDA;
+        err = launch_pdl(decode_down_ring_kernel, dim3(grid), dim3(DR_THREADS), size_t(RL.total), st, D, h, shp, W.nch,
+                         ids, weights, k, out);
+        if (err != cudaSuccess) {
+            (void)cudaGetLastError();
+            return DS4MOE_ECUDA;
+        }
+        return DS4MOE_OK;
+    }
     switch (wpl) {
 #define DN_CASE(V)                                                                                               \
     case V:                                                                                                      \

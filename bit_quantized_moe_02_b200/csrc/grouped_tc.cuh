@@ -8,8 +8,9 @@
 //               (kind::f16, fp32 accumulators in TMEM) for every K-chunk;
 //               tcgen05.commit releases the shared-memory stage back to the
 //               producers and finally signals the epilogue.
-//   warps 1-3   gather the tile's token rows (fp16 activations or SwiGLU
-//               outputs) with cp.async into 128B-swizzled K-major stages.
+//   warp 1      loads the tile's token rows (permuted fp16 activations or
+//               SwiGLU outputs, contiguous per expert) with one 2D TMA tensor
+//               copy per stage into a 128B-swizzled K-major stage.
 //   warps 4-11  stream the packed 2-bit (or 4-bit) blocks, dequantize them in
 //               registers (shared-memory codebook / sign-bit XOR / fp16 scale)
 //               and write fp16 tiles in the same swizzled K-major layout the
@@ -22,11 +23,15 @@
 // Every wait on an mbarrier is bounded; a timeout records DS4MOE_ETIMEOUT,
 // stops the CTA's roles and still frees TMEM before returning.
 #pragma once
+#include <cuda.h>
+
 #include "common.cuh"
 #include "grouped_mma.cuh"
 
 namespace ds4 {
 namespace tc {
+
+constexpr int FMT_F16 = 4;  // internal: dense fp16 rows used as they are (router weights)
 
 constexpr int M = 128;          // weight rows per accumulator
 constexpr int BK = 64;          // K per pipeline stage (one 128-byte swizzle row of fp16)
@@ -41,7 +46,7 @@ constexpr long long WAIT_NS = 2000000000LL;  // 2 s bound on any single wait
 
 template <bool GATEUP>
 struct Cfg {
-    static constexpr int STAGES = GATEUP ? 3 : 4;
+    static constexpr int STAGES = 4;
     static constexpr int STAGE = (GATEUP ? 2 : 1) * A_TILE + B_TILE;
     static constexpr int TMEM_COLS = GATEUP ? 256 : 128;
     static constexpr int TABLE_OFF = STAGES * STAGE;
@@ -141,6 +146,22 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// 2D TMA tensor load (tile mode, no multicast): box at (c0 = inner element, c1 = row) into shared memory,
+// completion counted on `bar`.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int c0, int c1, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+            dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
+        : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.release.cta.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(
+                     bar),
+                 "r"(bytes)
+                 : "memory");
+}
+
 __device__ __forceinline__ void cp_async_wait_le(int n) {
     // n is small and uniform; branch to the immediate forms
     if (n <= 0) asm volatile("cp.async.wait_group 0;" ::: "memory");
@@ -149,10 +170,172 @@ __device__ __forceinline__ void cp_async_wait_le(int n) {
     else asm volatile("cp.async.wait_group 3;" ::: "memory");
 }
 
+// ---- A producers: packed data for a "super-stage" of SS pipeline stages is loaded one super-stage ahead ------
+//
+// GATEUP: thread t owns matrix m = t / 128 (gate, up) and tile row R = t % 128 and writes all 64 weights of
+// its row per stage.  DOWN: thread t owns row R = t / 2 and half h = t % 2 (32 weights per stage).
+
+template <int AFMT, bool GATEUP>
+struct SPackCfg;
+template <> struct SPackCfg<DS4MOE_FMT_IQ2X, true> { static constexpr int SS = 4, NW = 18; };   // one super-block
+template <> struct SPackCfg<DS4MOE_FMT_Q4K, true> { static constexpr int SS = 2, NW = 20; };    // half super-block
+template <> struct SPackCfg<DS4MOE_FMT_BF16, true> { static constexpr int SS = 1, NW = 32; };
+template <> struct SPackCfg<DS4MOE_FMT_Q2K, false> { static constexpr int SS = 4, NW = 13; };
+template <> struct SPackCfg<DS4MOE_FMT_Q4K, false> { static constexpr int SS = 4, NW = 20; };
+template <> struct SPackCfg<DS4MOE_FMT_BF16, false> { static constexpr int SS = 1, NW = 16; };
+template <> struct SPackCfg<FMT_F16, false> { static constexpr int SS = 1, NW = 16; };
+
+template <int AFMT, bool GATEUP>
+struct SPack {
+    uint32_t w[SPackCfg<AFMT, GATEUP>::NW];
+};
+
+__device__ __forceinline__ void ld4(uint32_t *w, const uint8_t *p) {
+    const uint4 v = ldg_nc_v4(p);
+    w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+}
+
+// Load super-stage `ss` (K range [ss*SS*64, (ss+1)*SS*64)) of row `row` (half h for DOWN).
+template <int AFMT, bool GATEUP>
+__device__ __forceinline__ void sp_load(SPack<AFMT, GATEUP> &pk, const uint8_t *__restrict__ mat, const Planes &P,
+                                        int row, int h, int K, int ss) {
+    const int nsb = K / QK;
+    if constexpr (AFMT == DS4MOE_FMT_IQ2X) {  // GATEUP, super-block ss
+        const size_t b = size_t(row) * nsb + ss;
+        ld4(pk.w + 0, mat + P.off[0] + b * 32);
+        ld4(pk.w + 4, mat + P.off[0] + b * 32 + 16);
+        ld4(pk.w + 8, mat + P.off[1] + b * 32);
+        ld4(pk.w + 12, mat + P.off[1] + b * 32 + 16);
+        pk.w[16] = ldg_nc_u32(mat + P.off[2] + b * 4);
+        pk.w[17] = *reinterpret_cast<const uint16_t *>(mat + P.off[3] + b * 2);
+    } else if constexpr (AFMT == DS4MOE_FMT_Q4K && GATEUP) {  // half super-block ss
+        const size_t b = size_t(row) * nsb + ss / 2;
+        const uint8_t *q = mat + P.off[0] + b * 128 + (ss & 1) * 64;
+#pragma unroll
+        for (int i = 0; i < 4; i++) ld4(pk.w + 4 * i, q + 16 * i);
+        const uint32_t *sc = reinterpret_cast<const uint32_t *>(mat + P.off[1] + b * 12);
+        pk.w[16] = sc[0]; pk.w[17] = sc[1]; pk.w[18] = sc[2];
+        pk.w[19] = ldg_nc_u32(mat + P.off[2] + b * 4);
+    } else if constexpr (AFMT == DS4MOE_FMT_Q2K) {  // DOWN, super-block ss; stage j uses sub-blocks 4j+2h, +1
+        const size_t b = size_t(row) * nsb + ss;
+        const uint8_t *q = mat + P.off[0] + b * 64 + h * 8;
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+            const uint2 v = *reinterpret_cast<const uint2 *>(q + 16 * j);
+            pk.w[2 * j] = v.x; pk.w[2 * j + 1] = v.y;
+        }
+        ld4(pk.w + 8, mat + P.off[1] + b * 16);
+        pk.w[12] = ldg_nc_u32(mat + P.off[2] + b * 4);
+    } else if constexpr (AFMT == DS4MOE_FMT_Q4K) {  // DOWN, super-block ss; stage j uses sub-block 2j+h
+        const size_t b = size_t(row) * nsb + ss;
+#pragma unroll
+        for (int j = 0; j < 4; j++) ld4(pk.w + 4 * j, mat + P.off[0] + b * 128 + (2 * j + h) * 16);
+        const uint32_t *sc = reinterpret_cast<const uint32_t *>(mat + P.off[1] + b * 12);
+        pk.w[16] = sc[0]; pk.w[17] = sc[1]; pk.w[18] = sc[2];
+        pk.w[19] = ldg_nc_u32(mat + P.off[2] + b * 4);
+    } else {  // BF16 / F16 dense rows: one stage = 64 (GATEUP) or 32 (DOWN, half h) elements
+        const uint8_t *p = mat + (size_t(row) * K + size_t(ss) * BK + (GATEUP ? 0 : h * 32)) * 2;
+#pragma unroll
+        for (int i = 0; i < SPackCfg<AFMT, GATEUP>::NW / 4; i++) ld4(pk.w + 4 * i, p + 16 * i);
+    }
+}
+
+__device__ __forceinline__ void q4k_pairs(uint32_t word, __half2 a2, __half2 c2, uint4 &o) {
+    const __half2 k1024 = __float2half2_rn(1024.f);
+    __half2 P[4];
+#pragma unroll
+    for (int n = 0; n < 4; n++) {
+        const uint32_t v = ((word >> (4 * n)) & 0x000F000Fu) | 0x64006400u;
+        P[n] = __hfma2(__hsub2(u32_as_half2(v), k1024), a2, c2);  // (w_n, w_{n+4})
+    }
+    o.x = half2_as_u32(__lows2half2(P[0], P[1]));
+    o.y = half2_as_u32(__lows2half2(P[2], P[3]));
+    o.z = half2_as_u32(__highs2half2(P[0], P[1]));
+    o.w = half2_as_u32(__highs2half2(P[2], P[3]));
+}
+
+// Dequantize stage j (compile-time) of a super-stage: GATEUP -> 8 uint4 (64 weights), DOWN -> 4 uint4 (32).
+template <int AFMT, bool GATEUP, int J>
+__device__ __forceinline__ void sp_dequant(const SPack<AFMT, GATEUP> &pk, int h, int ss, const uint8_t *tbl_lane,
+                                           uint4 *o, bool &inf) {
+    constexpr uint32_t M = 0x80008000u;
+    if constexpr (AFMT == DS4MOE_FMT_IQ2X) {
+        const float dv = half_bits_to_float(uint16_t(pk.w[17]));
+#pragma unroll
+        for (int gg = 0; gg < 2; gg++) {
+            constexpr int dummy = 0;
+            (void)dummy;
+            const int g = 2 * J + gg;
+            const float s = float((pk.w[16] >> (4 * g)) & 15u);
+            const __half2 D2 = __float2half2_rn((dv * (0.5f + s)) * 0.25f);
+            const uint32_t W = pk.w[8 + g];
+#pragma unroll
+            for (int j = 0; j < 4; j++) {
+                const uint32_t ib = (pk.w[g] >> (8 * j)) & 0xFFu;
+                const uint4 cb = *reinterpret_cast<const uint4 *>(tbl_lane + ib * 128);
+                const uint32_t Wj = W << (4 * j);
+                uint4 &r = o[gg * 4 + j];
+                r.x = half2_as_u32(__hmul2(u32_as_half2(cb.x ^ (Wj & M)), D2));
+                r.y = half2_as_u32(__hmul2(u32_as_half2(cb.y ^ ((Wj << 1) & M)), D2));
+                r.z = half2_as_u32(__hmul2(u32_as_half2(cb.z ^ ((Wj << 2) & M)), D2));
+                r.w = half2_as_u32(__hmul2(u32_as_half2(cb.w ^ ((Wj << 3) & M)), D2));
+            }
+        }
+    } else if constexpr (AFMT == DS4MOE_FMT_Q4K) {
+        const float dv = half_bits_to_float(uint16_t(pk.w[19] & 0xFFFF));
+        const float dm = half_bits_to_float(uint16_t(pk.w[19] >> 16));
+        constexpr int NSUB = GATEUP ? 2 : 1;
+#pragma unroll
+        for (int u = 0; u < NSUB; u++) {
+            // sub-block within the super-block
+            const int sub = GATEUP ? ((ss & 1) * 4 + 2 * J + u) : (2 * J + h);
+            const int sc = q4k_field(pk.w[16], pk.w[17], pk.w[18], 6 * sub);
+            const int mn = q4k_field(pk.w[16], pk.w[17], pk.w[18], 48 + 6 * sub);
+            const __half2 a2 = __float2half2_rn(dv * float(sc));
+            const __half2 c2 = __float2half2_rn(-(dm * float(mn)));
+            const uint32_t *q = pk.w + (GATEUP ? (2 * J + u) * 4 : J * 4);
+#pragma unroll
+            for (int w = 0; w < 4; w++) q4k_pairs(q[w], a2, c2, o[u * 4 + w]);
+        }
+    } else if constexpr (AFMT == DS4MOE_FMT_Q2K) {
+        const float dv = half_bits_to_float(uint16_t(pk.w[12] & 0xFFFF));
+        const float dm = half_bits_to_float(uint16_t(pk.w[12] >> 16));
+        const __half2 k1024 = __float2half2_rn(1024.f);
+        const uint32_t scw = (pk.w[8 + J] >> (16 * h)) & 0xFFFFu;  // bytes of sub-blocks 4J+2h, 4J+2h+1
+#pragma unroll
+        for (int sb = 0; sb < 2; sb++) {
+            const uint32_t scb = (scw >> (8 * sb)) & 0xFFu;
+            const __half2 a2 = __float2half2_rn(dv * float(scb & 15u));
+            const __half2 c2 = __float2half2_rn(-(dm * float(scb >> 4)));
+            __half2 P[8];
+#pragma unroll
+            for (int p = 0; p < 8; p++) {
+                const uint32_t v = ((pk.w[2 * J + sb] >> (2 * p)) & 0x00030003u) | 0x64006400u;
+                P[p] = __hfma2(__hsub2(u32_as_half2(v), k1024), a2, c2);  // (w_p, w_{p+8})
+            }
+            uint32_t *oo = reinterpret_cast<uint32_t *>(&o[2 * sb]);
+#pragma unroll
+            for (int p = 0; p < 4; p++) {
+                oo[p] = half2_as_u32(__lows2half2(P[2 * p], P[2 * p + 1]));
+                oo[4 + p] = half2_as_u32(__highs2half2(P[2 * p], P[2 * p + 1]));
+            }
+        }
+    } else if constexpr (AFMT == FMT_F16) {
+#pragma unroll
+        for (int i = 0; i < SPackCfg<AFMT, GATEUP>::NW / 4; i++)
+            o[i] = make_uint4(pk.w[4 * i], pk.w[4 * i + 1], pk.w[4 * i + 2], pk.w[4 * i + 3]);
+    } else {  // BF16
+#pragma unroll
+        for (int i = 0; i < SPackCfg<AFMT, GATEUP>::NW / 4; i++)
+            o[i] = make_uint4(bf16x2_to_f16x2(pk.w[4 * i], inf), bf16x2_to_f16x2(pk.w[4 * i + 1], inf),
+                              bf16x2_to_f16x2(pk.w[4 * i + 2], inf), bf16x2_to_f16x2(pk.w[4 * i + 3], inf));
+    }
+}
+
 // ---- the kernel -------------------------------------------------------------------------------------------
 
 template <int AFMT, bool GATEUP>
-__global__ void __launch_bounds__(THREADS, 1) grouped_tc_kernel(GroupedArgs a) {
+__global__ void __launch_bounds__(THREADS, 1) grouped_tc_kernel(GroupedArgs a, const __grid_constant__ CUtensorMap tmap_b) {
     using C = Cfg<GATEUP>;
     constexpr int S = C::STAGES;
     extern __shared__ uint8_t smem_raw[];
@@ -161,7 +344,6 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_tc_kernel(GroupedArgs a) {
     __shared__ __align__(8) uint64_t bars[3 * 4 + 1];  // full_a[S], full_b[S], empty[S], accum
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
-    __shared__ int32_t s_brow[NT];
     __shared__ float s_colsc[NT];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -188,7 +370,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_tc_kernel(GroupedArgs a) {
     if (tid == 0) {
         for (int s = 0; s < S; s++) {
             mbar_init(full_a(s), N_WA);
-            mbar_init(full_b(s), N_WB);
+            mbar_init(full_b(s), 1);
             mbar_init(empty(s), 1);
         }
         mbar_init(accum_bar, 1);
@@ -200,15 +382,13 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_tc_kernel(GroupedArgs a) {
         tc_fence_before();
     }
     if (tid < NT) {
+        // per-token column scale: the activation's power-of-two scale (indexed by token) times the gate weight
         float sc = 1.f;
-        int brow = 0;
         if (tid < cnt) {
             const int pos = pos0 + tid;
-            brow = a.b_rowidx ? a.b_rowidx[pos] : pos;
-            if (a.b_colscale) sc *= a.b_colscale[brow];
+            if (a.b_colscale) sc *= a.b_colscale[a.b_rowidx ? a.b_rowidx[pos] : pos];
             if (a.pos_weight) sc *= a.pos_weight[pos];
         }
-        s_brow[tid] = brow;
         s_colsc[tid] = sc;
     }
     if constexpr (AFMT == DS4MOE_FMT_IQ2X) {
@@ -251,69 +431,86 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_tc_kernel(GroupedArgs a) {
         }
         __syncwarp();
     } else if (warp < W_B0 + N_WB) {
-        // ------------------------------------------------------------------ token-row loaders (cp.async)
-        const int bt = tid - W_B0 * 32;  // 0 .. 95
-        const uint8_t *bsrc = reinterpret_cast<const uint8_t *>(a.b_src);
-        const int nrow = cnt;
-        int lag_arrive = 0;  // next stage index whose arrival is pending
-        for (int kc = 0; kc < nk; kc++) {
-            const int s = kc % S;
-            const uint32_t par = ((kc / S) & 1) ^ 1;
-            if (!mbar_wait(empty(s), par, abort_flag)) break;
-            const uint32_t bst = smem_u32(smem + s * C::STAGE + (GATEUP ? 2 : 1) * A_TILE);
-            for (int job = bt; job < nrow * 8; job += N_WB * 32) {
-                const int n = job >> 3, c = job & 7;
-                cp_async16(bst + swz(n, c), bsrc + (size_t(s_brow[n]) * a.K + kc * BK + c * 8) * 2, 16);
+        // ------------------------------------------------------------------ token rows: one 2D TMA copy per stage
+        if (warp == W_B0 && lane == 0) {
+            int issued = 0;
+            for (int kc = 0; kc < nk; kc++) {
+                const int s = kc % S;
+                const uint32_t par = ((kc / S) & 1) ^ 1;
+                if (!mbar_wait(empty(s), par, abort_flag)) break;
+                const uint32_t bst = smem_u32(smem + s * C::STAGE + (GATEUP ? 2 : 1) * A_TILE);
+                mbar_expect_tx(full_b(s), B_TILE);  // full 128-row box, rows past the tensor are zero-filled
+                tma_load_2d(bst, &tmap_b, kc * BK, pos0, full_b(s));
+                issued = kc + 1;
             }
-            cp_async_commit();
-            if (kc - lag_arrive >= S - 1) {
-                cp_async_wait_le(S - 1);
-                fence_proxy_async();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(full_b(lag_arrive % S));
-                lag_arrive++;
+            if (*abort_flag) {
+                // let this CTA's copies still in flight land before its shared memory is released (bounded)
+                const uint64_t t0 = globaltimer();
+                for (int kc = max(0, issued - S); kc < issued; kc++)
+                    while (!mbar_try_wait(full_b(kc % S), (kc / S) & 1) && globaltimer() - t0 < uint64_t(WAIT_NS)) {
+                    }
             }
         }
-        cp_async_wait_le(0);
-        fence_proxy_async();
         __syncwarp();
-        for (; lag_arrive < nk; lag_arrive++)
-            if (lane == 0) mbar_arrive(full_b(lag_arrive % S));
     } else {
         // ------------------------------------------------------------------ dequantizing producers
+        constexpr int SS = SPackCfg<AFMT, GATEUP>::SS;
+        constexpr int NOUT = GATEUP ? 8 : 4;
         const int at = tid - W_A0 * 32;  // 0 .. 255
-        const int R = at >> 1, hh = at & 1;
-        const uint8_t *mat0 = a.a0 + size_t(e) * a.a_stride;
-        const uint8_t *mat1 = GATEUP ? a.a1 + size_t(e) * a.a_stride : nullptr;
-        const int row = (GATEUP ? blockIdx.x * M : blockIdx.x * M) + R;
+        const int m = GATEUP ? at >> 7 : 0;
+        const int R = GATEUP ? at & 127 : at >> 1;
+        const int h = GATEUP ? 0 : at & 1;
+        const uint8_t *mat = (GATEUP && m ? a.a1 : a.a0) + size_t(e) * a.a_stride;
+        const int row = blockIdx.x * M + R;
         const uint8_t *tbl_lane = tbl + (lane & 7) * 16;
-        APack p0, p1;
-        a_load<AFMT>(p0, mat0, a.pa, row, a.K, hh * 32);
-        if constexpr (GATEUP) a_load<AFMT>(p1, mat1, a.pa, row, a.K, hh * 32);
-        for (int kc = 0; kc < nk; kc++) {
-            const int s = kc % S;
-            const uint32_t par = ((kc / S) & 1) ^ 1;
-            if (!mbar_wait(empty(s), par, abort_flag)) break;
-            uint8_t *ast = smem + s * C::STAGE;
-            uint4 o[4];
-            bool inf = false;
-            a_dequant<AFMT, 128>(p0, tbl_lane, kc * BK + hh * 32, o, inf);
+        const int nss = nk / SS;
+        // packed data of PF super-stages is in flight: super-stage ss+PF-1 is requested while ss is consumed
+        constexpr int PF = SPackCfg<AFMT, GATEUP>::NW <= 20 ? 3 : 2;
+        SPack<AFMT, GATEUP> pf[PF];
 #pragma unroll
-            for (int j = 0; j < 4; j++) *reinterpret_cast<uint4 *>(ast + swz(R, hh * 4 + j)) = o[j];
-            if constexpr (GATEUP) {
-                a_dequant<AFMT, 128>(p1, tbl_lane, kc * BK + hh * 32, o, inf);
+        for (int p = 0; p < PF - 1; p++)
+            if (p < nss) sp_load<AFMT, GATEUP>(pf[p], mat, a.pa, row, h, a.K, p);
+        bool inf = false;
+        bool run = true;
+        for (int base = 0; base < nss && run; base += PF) {
 #pragma unroll
-                for (int j = 0; j < 4; j++) *reinterpret_cast<uint4 *>(ast + A_TILE + swz(R, hh * 4 + j)) = o[j];
+            for (int q = 0; q < PF; q++) {
+                const int ss = base + q;
+                if (ss >= nss || !run) break;
+                if (ss + PF - 1 < nss) sp_load<AFMT, GATEUP>(pf[(q + PF - 1) % PF], mat, a.pa, row, h, a.K, ss + PF - 1);
+                const SPack<AFMT, GATEUP> &cur = pf[q];
+#pragma unroll
+                for (int jj = 0; jj < SS; jj++) {
+                    const int kc = ss * SS + jj;
+                    const int s = kc % S;
+                    const uint32_t par = ((kc / S) & 1) ^ 1;
+                    if (!mbar_wait(empty(s), par, abort_flag)) {
+                        run = false;
+                        break;
+                    }
+                    uint4 o[NOUT];
+                    if constexpr (SS == 4) {
+                        if (jj == 0) sp_dequant<AFMT, GATEUP, 0>(cur, h, ss, tbl_lane, o, inf);
+                        else if (jj == 1) sp_dequant<AFMT, GATEUP, 1>(cur, h, ss, tbl_lane, o, inf);
+                        else if (jj == 2) sp_dequant<AFMT, GATEUP, 2>(cur, h, ss, tbl_lane, o, inf);
+                        else sp_dequant<AFMT, GATEUP, 3>(cur, h, ss, tbl_lane, o, inf);
+                    } else if constexpr (SS == 2) {
+                        if (jj == 0) sp_dequant<AFMT, GATEUP, 0>(cur, h, ss, tbl_lane, o, inf);
+                        else sp_dequant<AFMT, GATEUP, 1>(cur, h, ss, tbl_lane, o, inf);
+                    } else {
+                        sp_dequant<AFMT, GATEUP, 0>(cur, h, ss, tbl_lane, o, inf);
+                    }
+                    uint8_t *ast = smem + s * C::STAGE + m * A_TILE;
+#pragma unroll
+                    for (int c = 0; c < NOUT; c++)
+                        *reinterpret_cast<uint4 *>(ast + swz(R, (GATEUP ? 0 : h * 4) + c)) = o[c];
+                    fence_proxy_async();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(full_a(s));
+                }
             }
-            if (inf) set_device_error(DS4MOE_EDEVICE);
-            if (kc + 1 < nk) {
-                a_load<AFMT>(p0, mat0, a.pa, row, a.K, (kc + 1) * BK + hh * 32);
-                if constexpr (GATEUP) a_load<AFMT>(p1, mat1, a.pa, row, a.K, (kc + 1) * BK + hh * 32);
-            }
-            fence_proxy_async();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(full_a(s));
         }
+        if (inf) set_device_error(DS4MOE_EDEVICE);
 
         // ------------------------------------------------------------------ epilogue (warps 4..7)
         if (warp < W_A0 + 4) {

@@ -47,6 +47,18 @@ __global__ void __launch_bounds__(256) prep_x_kernel(const __nv_bfloat16 *__rest
     }
 }
 
+// Permuted activations for the routed gate/up GEMM: x_perm[p] = x16[perm_tok[p]], so that every expert's
+// token rows are contiguous and one tensor copy moves a whole token tile.  One warp per row.
+__global__ void __launch_bounds__(256) gather_rows_kernel(const __half *__restrict__ x16, int d,
+                                                          const int32_t *__restrict__ perm_tok, int N,
+                                                          __half *__restrict__ x_perm) {
+    const int p = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+    if (p >= N) return;
+    const uint4 *src = reinterpret_cast<const uint4 *>(x16 + size_t(perm_tok[p]) * d);
+    uint4 *dst = reinterpret_cast<uint4 *>(x_perm + size_t(p) * d);
+    for (int i = lane; i < d / 8; i += 32) dst[i] = src[i];
+}
+
 // Per-block expert histogram of the T*k routed pairs.
 __global__ void __launch_bounds__(PERM_BLOCK) perm_count_kernel(const int32_t *__restrict__ ids, int N, int E,
                                                                 int32_t *__restrict__ blk_counts) {

@@ -25,6 +25,7 @@ __global__ void __launch_bounds__(256) route_logits_small_kernel(const __nv_bflo
     if (e < E) {
         int kq = d / 4;  // multiple of 64
         const __half *row = wr + size_t(e) * d + q * kq;
+#pragma unroll 4
         for (int c = lane * 8; c < kq; c += 256) {
             uint4 wv = *reinterpret_cast<const uint4 *>(row + c);
             float wf[8];
@@ -66,7 +67,7 @@ __global__ void __launch_bounds__(256) route_logits_small_kernel(const __nv_bflo
     }
 }
 
-// ---- large T (prefill): 64 tokens x 64 experts per CTA, K chunks of 32.
+// ---- large T without a tensor-core tiling (E not a multiple of 128): 64 tokens x 64 experts per CTA.
 __global__ void __launch_bounds__(256) route_logits_tiled_kernel(const __nv_bfloat16 *__restrict__ x, int T, int d,
                                                                  const __half *__restrict__ wr,
                                                                  const float *__restrict__ bias, int E,
@@ -125,21 +126,24 @@ __global__ void __launch_bounds__(256) route_logits_tiled_kernel(const __nv_bflo
     }
 }
 
-// ---- top-k: one warp per token, E <= 1024 logits spread over the lanes.
+// ---- top-k: one warp per token, E <= 32 * PER logits spread over the lanes.
+// late_bias: added here when the logits kernel did not add it (tensor-core path), else NULL.
+template <int PER>
 __global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict__ logits, int T, int E, int k,
+                                                         const float *__restrict__ late_bias,
                                                          int32_t *__restrict__ ids, float *__restrict__ weights) {
     int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
     if (warp >= T) return;
     const float *lg = logits + size_t(warp) * E;
-    float v[32];
+    float v[PER];
     uint32_t taken = 0;
-    int per = (E + 31) / 32;
 #pragma unroll
-    for (int i = 0; i < 32; i++) v[i] = (i < per && lane + 32 * i < E) ? lg[lane + 32 * i] : -INFINITY;
+    for (int i = 0; i < PER; i++)
+        v[i] = (lane + 32 * i < E) ? lg[lane + 32 * i] + (late_bias ? late_bias[lane + 32 * i] : 0.f) : -INFINITY;
     uint32_t valid = 0;
 #pragma unroll
-    for (int i = 0; i < 32; i++)
-        if (i < per && lane + 32 * i < E) valid |= 1u << i;
+    for (int i = 0; i < PER; i++)
+        if (lane + 32 * i < E) valid |= 1u << i;
     float ssum = 0.f, s_mine = 0.f;
     int id_mine = -1;
     for (int j = 0; j < k; j++) {
@@ -147,7 +151,7 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict
         float bv = -INFINITY;
         int bid = 0x7fffffff;
 #pragma unroll
-        for (int i = 0; i < 32; i++) {
+        for (int i = 0; i < PER; i++) {
             bool ok = ((valid & ~taken) >> i) & 1u;
             if (ok && (v[i] > bv || bid == 0x7fffffff)) { bv = v[i]; bid = lane + 32 * i; }
         }
