@@ -1,0 +1,599 @@
+// Single-token decode: GEMV over the k selected experts' packed rows and the
+// shared expert's bf16 rows, SwiGLU, and the weighted combine, in two kernels
+// (gate/up, then down + combine), each one persistent CTA of 16 warps per SM.
+//
+// Work is cut into warp-sized units of a few rows (8 gate/up row pairs, or 2
+// output rows of the down projection over all k experts).  The 32 lanes of a
+// warp split the contraction dimension: in each pass every lane owns a fixed
+// slice, holds that slice of the activations in registers (loaded once per
+// pass from shared memory) and walks the unit's rows, so consecutive lanes read
+// consecutive bytes of a row's packed planes (coalesced) and the only shared-
+// memory stream per weight is the dequantization table.  The packed data of
+// the next few rows is kept in flight in a small register ring.  A unit ends
+// with one butterfly reduce-scatter of its row sums over the 32 lanes: no
+// partial sums leave the SM and the summation order is fixed.
+//
+//  * gate/up (IQ2X): codebook table in shared memory with 16 lane slots per
+//    entry (128-bit lookups without bank conflicts, addressed with one byte
+//    permute); signs XORed onto the fp16 sign bits; packed fp16 FMAs inside a
+//    32-weight group (one scale), fp32 across groups; the row's first lane
+//    writes h_j = silu(g) * u.  Shared-expert row pairs are units as well and
+//    run before the grid-dependency wait (they need neither ids nor the router).
+//  * down (Q2K): byte -> 4 x fp16 table (32 lane slots); h_j staged per expert
+//    as fp16 scaled by a power of two, with sums of every 8 staged values for
+//    the min term; a unit is 2 output rows over all k experts and the shared
+//    expert, accumulated as out[r] = sum_j w_j (D_j h_j)[r] + (Ds hs)[r].
+//
+// The method (routed experts quantized, IQ2_XXS-style gate/up, Q2_K-style
+// down, shared expert unquantized) is the ds4 news summary's "model weights"
+// section; the kernel design is this library's own.
+#pragma once
+#include "common.cuh"
+
+namespace ds4 {
+
+struct ExpertsDev {
+    int d, f, E, fs;
+    int fmt_gate, fmt_down;
+    const uint8_t *gate, *up, *down;
+    uint64_t gate_stride, up_stride, down_stride;
+    const uint8_t *codebook;
+    const __nv_bfloat16 *sh_gate, *sh_up, *sh_down;
+    Planes pg;  // planes of one gate/up matrix [f x d]
+    Planes pd;  // planes of one down matrix [d x f]
+};
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+    return v;
+}
+__device__ __forceinline__ uint2 lds64(uint32_t addr) {
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+    return v;
+}
+__device__ __forceinline__ uint2 ldg_nc_v2(const void *p) {
+    uint2 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(p));
+    return r;
+}
+__device__ __forceinline__ uint32_t ldg_nc_u16(const void *p) {
+    unsigned short r;
+    asm volatile("ld.global.nc.L1::no_allocate.u16 %0, [%1];" : "=h"(r) : "l"(p));
+    return r;
+}
+__device__ __forceinline__ uint32_t ldg_nc_u8(const void *p) {
+    unsigned short r;
+    asm volatile("ld.global.nc.L1::no_allocate.u8 %0, [%1];" : "=h"(r) : "l"(p));
+    return r & 0xFFu;
+}
+
+// Fire-and-forget bulk prefetch of [p, p + bytes) into L2 (16-byte aligned address and size).  A warp issues
+// these for its next unit, so the bytes in flight are not limited by the registers that hold loaded data.
+__device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+
+// Staged activations are stored in 16-byte chunks at swizzled positions: chunk c at c ^ ((c >> 3) & 7).  A lane
+// that reads its slice of 1, 2, 4 or 8 consecutive chunks (lane stride 16 to 128 bytes) then meets no bank
+// conflict within a quarter-warp.
+__host__ __device__ __forceinline__ int swz16(int c) { return c ^ ((c >> 3) & 7); }
+
+// Butterfly reduce-scatter over the 32 lanes of 16 per-lane partial sums: afterwards lanes 2v and 2v+1 both
+// hold the full sum of value v = (lane >> 1) & 15.
+__device__ __forceinline__ float reduce16(float (&v)[16], int lane) {
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+        const bool hi = lane & 16;
+        const float send = hi ? v[i] : v[i + 8], keep = hi ? v[i + 8] : v[i];
+        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        const bool hi = lane & 8;
+        const float send = hi ? v[i] : v[i + 4], keep = hi ? v[i + 4] : v[i];
+        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+    }
+#pragma unroll
+    for (int i = 0; i < 2; i++) {
+        const bool hi = lane & 4;
+        const float send = hi ? v[i] : v[i + 2], keep = hi ? v[i + 2] : v[i];
+        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+    }
+    const bool hi = lane & 2;
+    float r = (hi ? v[1] : v[0]) + __shfl_xor_sync(0xffffffffu, hi ? v[0] : v[1], 2);
+    return r + __shfl_xor_sync(0xffffffffu, r, 1);
+}
+
+// ============================================================================ gate / up
+
+constexpr int DG_WARPS = 16;
+constexpr int DG_THREADS = DG_WARPS * 32;
+constexpr uint32_t DG_TABLE_ABS = 0x10000;  // absolute shared address of the 64 KB codebook table
+constexpr int DG_ROWS = 8;                  // gate/up row pairs per unit (routed and shared)
+constexpr int DG_MAX_D = 8192;
+
+// Contraction lengths the gate/up kernel takes: d = 256 * nblk with nblk in {1, 2, 4, 8, 16, 32}.  A lane owns
+// VPP = min(nblk, 8) consecutive 8-vectors of a row per pass; nblk / VPP passes.
+__host__ __device__ __forceinline__ bool dg_supported_d(int d) {
+    const int nblk = d / QK;
+    return d % QK == 0 && nblk >= 1 && nblk <= 32 && (nblk & (nblk - 1)) == 0;
+}
+// dynamic shared memory: everything up to the table's end, then x as fp16 (2d bytes) and fp32 (4d bytes)
+__host__ __device__ __forceinline__ int dg_smem_bytes(int d) { return int(DG_TABLE_ABS) + 65536 + d * 6; }
+
+template <int VPP>
+struct IqRp {  // a lane's slice of one IQ2X row in one pass: VPP 8-vectors
+    static constexpr int NW = (VPP + 3) / 4;
+    uint32_t idx[NW];  // codebook indices, one byte per vector
+    uint32_t sgn[NW];  // sign words of the groups the slice touches
+    uint32_t scl, d;   // the block's 4-bit group scales and fp16 scale
+};
+
+// v0: first vector of the slice within the row (a multiple of VPP)
+template <int VPP>
+__device__ __forceinline__ void iq_rp_load(IqRp<VPP> &R, const uint8_t *W, const Planes &P, size_t row, int nblk,
+                                           int v0) {
+    const size_t rb = row * size_t(nblk) * 32;  // bytes of one row in the index and sign planes
+    const uint8_t *ip = W + P.off[0] + rb + v0;
+    const uint8_t *sp = W + P.off[1] + rb + (v0 & ~3);
+    if constexpr (VPP == 8) {
+        const uint2 a = ldg_nc_v2(ip), b = ldg_nc_v2(sp);
+        R.idx[0] = a.x; R.idx[1] = a.y; R.sgn[0] = b.x; R.sgn[1] = b.y;
+    } else {
+        R.idx[0] = VPP == 4 ? ldg_nc_u32(ip) : VPP == 2 ? ldg_nc_u16(ip) : ldg_nc_u8(ip);
+        R.sgn[0] = ldg_nc_u32(sp);
+    }
+    const size_t blk = row * size_t(nblk) + v0 / 32;
+    R.scl = ldg_nc_u32(W + P.off[2] + blk * 4);
+    R.d = ldg_nc_u16(W + P.off[3] + blk * 2);
+}
+
+// Dot product of a lane's row slice with its activations xr (fp16 pairs, VPP vectors).  Group g of a block
+// (vectors 4g..4g+3) has weights (d * (0.5 + s_g) / 4) * grid * sign; fp16 FMAs inside a group, fp32 across.
+template <int VPP>
+__device__ __forceinline__ float iq_rp_dot(const IqRp<VPP> &R, const uint4 (&xr)[VPP], int v0, uint32_t lane_tbl) {
+    constexpr uint32_t M = 0x80008000u;
+    constexpr int NG = VPP >= 4 ? VPP / 4 : 1, VG = VPP >= 4 ? 4 : VPP;
+    const int pos0 = v0 & 3;          // position of the first vector inside its group (0 when VPP >= 4)
+    const int g0 = (v0 >> 2) & 7;     // group of the first vector inside its block
+    const float dv = half_bits_to_float(uint16_t(R.d));
+    const float d4 = dv * 0.25f, d8 = dv * 0.125f;
+    float acc = 0.f;
+#pragma unroll
+    for (int g = 0; g < NG; g++) {
+        const uint32_t W = R.sgn[g];
+        __half2 a0 = __float2half2_rn(0.f), a1 = a0;
+#pragma unroll
+        for (int j = 0; j < VG; j++) {
+            const int v = g * 4 + j;
+            const uint4 cb = lds128(__byte_perm(R.idx[v >> 2], lane_tbl, 0x7604 | ((v & 3) << 4)));
+            const uint32_t Wj = W << (4 * (pos0 + j));
+            a0 = __hfma2(u32_as_half2(cb.x ^ (Wj & M)), u32_as_half2(xr[v].x), a0);
+            a1 = __hfma2(u32_as_half2(cb.y ^ ((Wj << 1) & M)), u32_as_half2(xr[v].y), a1);
+            a0 = __hfma2(u32_as_half2(cb.z ^ ((Wj << 2) & M)), u32_as_half2(xr[v].z), a0);
+            a1 = __hfma2(u32_as_half2(cb.w ^ ((Wj << 3) & M)), u32_as_half2(xr[v].w), a1);
+        }
+        const float Dg = fmaf(float((R.scl >> (4 * (g0 + g))) & 15u), d4, d8);  // d * (0.5 + s) / 4, exact
+        const float2 fa = __half22float2(__hadd2(a0, a1));
+        acc = fmaf(Dg, fa.x + fa.y, acc);
+    }
+    return acc;
+}
+
+__device__ __forceinline__ float bf16x8_dot(const uint4 w, const float4 a, const float4 b) {
+    float s = bf16_lo(w.x) * a.x;
+    s = fmaf(bf16_hi(w.x), a.y, s);
+    s = fmaf(bf16_lo(w.y), a.z, s);
+    s = fmaf(bf16_hi(w.y), a.w, s);
+    s = fmaf(bf16_lo(w.z), b.x, s);
+    s = fmaf(bf16_hi(w.z), b.y, s);
+    s = fmaf(bf16_lo(w.w), b.z, s);
+    s = fmaf(bf16_hi(w.w), b.w, s);
+    return s;
+}
+
+// Units: shared-expert units first (rows 8u .. 8u+7 of Gs, Us), then routed units (expert slot j, rows
+// 8i .. 8i+7).  Row-matrix index rr = 2 * (row - first row) + (0 gate, 1 up).
+template <int VPP>
+__global__ void __launch_bounds__(DG_THREADS, 1)
+    decode_gateup_kernel(const ExpertsDev ex, const __nv_bfloat16 *__restrict__ x, const int32_t *__restrict__ ids,
+                         int k, float *__restrict__ h_out, float *__restrict__ hs_out) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    __shared__ float s_red[DG_WARPS];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int d = ex.d, f = ex.f, fs = ex.fs;
+    const int nblk = d / QK;
+    const int npass = nblk / VPP;
+    const uint32_t sbase = smem_u32(smem);
+    uint8_t *tbl = smem + (DG_TABLE_ABS - sbase);
+    __half *x16 = reinterpret_cast<__half *>(tbl + 65536);
+    float *x32 = reinterpret_cast<float *>(tbl + 65536 + d * 2);
+    const uint32_t x16_s = DG_TABLE_ABS + 65536;
+
+    const int n_sh = fs / DG_ROWS;
+    const int upe = f / DG_ROWS;  // routed units per expert
+    const int n_all = n_sh + k * upe;
+    const int nW = gridDim.x * DG_WARPS;
+    const int u_first = warp * gridDim.x + blockIdx.x;
+    // the shared expert's rows of this warp's first unit go to L2 while the tables are built
+    if (u_first < n_sh && lane < 2 * DG_ROWS)
+        prefetch_l2((lane & 1 ? ex.sh_up : ex.sh_gate) + size_t(u_first * DG_ROWS + (lane >> 1)) * d, uint32_t(d * 2));
+
+    // prologue, one global round trip: every thread loads its codebook entry and its 8 activations together,
+    // then writes the codebook table (entry e, lane slot s at DG_TABLE_ABS + e * 256 + s * 16: 8 grid values as
+    // fp16), the fp32 activations, and after the block-wide max the fp16 activations scaled by the power of two
+    // that puts max |x| in [32, 64)
+    const int e_cb = tid >> 1;
+    const uint2 raw = *reinterpret_cast<const uint2 *>(ex.codebook + e_cb * 8);
+    constexpr int XPT = DG_MAX_D / (DG_THREADS * 8);  // 8-element activation chunks per thread (at most)
+    uint4 xv[XPT];
+#pragma unroll
+    for (int c = 0; c < XPT; c++) {
+        const int i = (tid + c * DG_THREADS) * 8;
+        if (i < d) xv[c] = *reinterpret_cast<const uint4 *>(x + i);
+    }
+    {
+        const uint32_t b[2] = {raw.x, raw.y};
+        __half2 hv[4];
+#pragma unroll
+        for (int p = 0; p < 4; p++)
+            hv[p] = __floats2half2_rn(float((b[p >> 1] >> (16 * (p & 1))) & 0xFF),
+                                      float((b[p >> 1] >> (16 * (p & 1) + 8)) & 0xFF));
+        const uint4 v = *reinterpret_cast<uint4 *>(hv);
+#pragma unroll
+        for (int s = 0; s < 8; s++) *reinterpret_cast<uint4 *>(tbl + e_cb * 256 + ((tid & 1) * 8 + s) * 16) = v;
+    }
+    float m = 0.f;
+#pragma unroll
+    for (int c = 0; c < XPT; c++) {
+        const int i = (tid + c * DG_THREADS) * 8;
+        if (i < d) {
+            const uint4 v = xv[c];
+            const float4 a = make_float4(bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y));
+            const float4 cc = make_float4(bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w));
+            reinterpret_cast<float4 *>(x32)[swz16(i / 4)] = a;
+            reinterpret_cast<float4 *>(x32)[swz16(i / 4 + 1)] = cc;
+            m = fmaxf(m, fmaxf(fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(a.z), fabsf(a.w))),
+                               fmaxf(fmaxf(fabsf(cc.x), fabsf(cc.y)), fmaxf(fabsf(cc.z), fabsf(cc.w)))));
+        }
+    }
+    m = warp_max(m);
+    if (lane == 0) s_red[warp] = m;
+    __syncthreads();
+    m = warp_max(lane < DG_WARPS ? s_red[lane] : 0.f);
+    const int xe = pow2_exponent_for(m, 6);
+    const float xs = ldexpf(1.f, xe), inv_xs = ldexpf(1.f, -xe);
+#pragma unroll
+    for (int c = 0; c < XPT; c++) {
+        const int i = (tid + c * DG_THREADS) * 8;
+        if (i < d) {
+            const uint4 v = xv[c];
+            reinterpret_cast<uint4 *>(x16)[swz16(i / 8)] =
+                make_uint4(half2_as_u32(__floats2half2_rn(bf16_lo(v.x) * xs, bf16_hi(v.x) * xs)),
+                           half2_as_u32(__floats2half2_rn(bf16_lo(v.y) * xs, bf16_hi(v.y) * xs)),
+                           half2_as_u32(__floats2half2_rn(bf16_lo(v.z) * xs, bf16_hi(v.z) * xs)),
+                           half2_as_u32(__floats2half2_rn(bf16_lo(v.w) * xs, bf16_hi(v.w) * xs)));
+        }
+    }
+    __syncthreads();
+
+    const uint32_t lane_tbl = DG_TABLE_ABS | uint32_t((lane & 15) * 16);
+    bool waited = false;
+    for (int u = u_first; u < n_all; u += nW) {
+        float acc[16];
+#pragma unroll
+        for (int i = 0; i < 16; i++) acc[i] = 0.f;
+        if (u < n_sh) {
+            // shared expert (bf16): pass p covers elements [256 p, 256 p + 256), lane slice 8 elements; ring of 8 rows
+            const size_t r0 = size_t(u) * DG_ROWS;
+            const int ns = d / 256, T = ns * 16;
+            auto wptr = [&](int t) {
+                const int rr = t & 15;
+                return (rr & 1 ? ex.sh_up : ex.sh_gate) + (r0 + (rr >> 1)) * d + (t >> 4) * 256 + lane * 8;
+            };
+            uint4 ring[8];
+#pragma unroll
+            for (int s = 0; s < 8; s++) ring[s] = ldg_nc_v4(wptr(s));
+            for (int p = 0; p < ns; p++) {
+                const float4 xa = reinterpret_cast<const float4 *>(x32)[swz16(p * 64 + 2 * lane)];
+                const float4 xb = reinterpret_cast<const float4 *>(x32)[swz16(p * 64 + 2 * lane + 1)];
+#pragma unroll
+                for (int rr = 0; rr < 16; rr++) {
+                    acc[rr] += bf16x8_dot(ring[rr & 7], xa, xb);
+                    const int tn = p * 16 + rr + 8;
+                    if (tn < T) ring[rr & 7] = ldg_nc_v4(wptr(tn));
+                }
+            }
+            const float v = reduce16(acc, lane);
+            const float up = __shfl_xor_sync(0xffffffffu, v, 2);  // lanes 4i: gate of row i; 4i + 2: up
+            if ((lane & 3) == 0) hs_out[r0 + (lane >> 2)] = silu(v) * up;
+            continue;
+        }
+        if (!waited) {
+            pdl_wait();  // ids come from the router
+            waited = true;
+        }
+        const int uu = u - n_sh;
+        const int j = uu / upe;
+        const size_t r0 = size_t(uu % upe) * DG_ROWS;
+        const int e = ids[j];
+        if (e < 0 || e >= ex.E) {
+            if (lane == 0) set_device_error(DS4MOE_EDEVICE);
+            continue;
+        }
+        const uint8_t *G = ex.gate + size_t(e) * ex.gate_stride, *U = ex.up + size_t(e) * ex.up_stride;
+        const int T = npass * 16;
+        auto load = [&](IqRp<VPP> &R, int t) {
+            const int rr = t & 15;
+            iq_rp_load<VPP>(R, rr & 1 ? U : G, ex.pg, r0 + (rr >> 1), nblk, (t >> 4) * 32 * VPP + lane * VPP);
+        };
+        IqRp<VPP> ring[4];
+#pragma unroll
+        for (int s = 0; s < 4; s++) load(ring[s], s);
+        for (int p = 0; p < npass; p++) {
+            const int v0 = p * 32 * VPP + lane * VPP;
+            uint4 xr[VPP];
+#pragma unroll
+            for (int v = 0; v < VPP; v++) xr[v] = lds128(x16_s + swz16(v0 + v) * 16);
+#pragma unroll
+            for (int rr = 0; rr < 16; rr++) {
+                acc[rr] += iq_rp_dot<VPP>(ring[rr & 3], xr, v0, lane_tbl);
+                const int tn = p * 16 + rr + 4;
+                if (tn < T) load(ring[rr & 3], tn);
+            }
+        }
+        const float v = reduce16(acc, lane);
+        const float up = __shfl_xor_sync(0xffffffffu, v, 2);
+        if ((lane & 3) == 0) h_out[size_t(j) * f + r0 + (lane >> 2)] = silu(v * inv_xs) * (up * inv_xs);
+    }
+}
+
+// ============================================================================ down + combine
+
+constexpr int DD_WARPS = 16;
+constexpr int DD_THREADS = DD_WARPS * 32;
+constexpr uint32_t DD_TABLE_ABS = 0x10000;  // absolute shared address of the 64 KB byte table
+constexpr int DD_ROWS = 2;                  // output rows per unit
+
+// Contraction lengths (f) the down kernel takes: f = 256 * 2^i up to 8192.  A lane owns EPL = min(64, f / 32)
+// consecutive weights of a row per pass; f / (32 EPL) passes.
+__host__ __device__ __forceinline__ bool dd_supported_f(int f) {
+    const int nblk = f / QK;
+    return f % QK == 0 && nblk >= 1 && nblk <= 32 && (nblk & (nblk - 1)) == 0;
+}
+
+struct DownSmemLayout {
+    int hq, hsum, hs, wsc, eid, total;  // byte offsets from the table base; total = dynamic bytes to request
+};
+__host__ __device__ __forceinline__ DownSmemLayout dd_layout(int k, int f, int fs) {
+    DownSmemLayout L;
+    L.hq = 65536;                                   // k x f fp16: h_j * 2^e_j
+    L.hsum = L.hq + k * f * 2;                      // k x f/8 floats: sums of 8 consecutive staged values
+    L.hs = L.hsum + ((k * (f / 8) * 4 + 15) & ~15);  // fs floats: shared-expert h
+    L.wsc = L.hs + ((fs * 4 + 15) & ~15);           // k floats: w_j * 2^-e_j
+    L.eid = L.wsc + ((k * 4 + 15) & ~15);           // k ints: expert ids
+    L.total = int(DD_TABLE_ABS) + L.eid + ((k * 4 + 15) & ~15);
+    return L;
+}
+
+template <int EPL>
+struct QkRp {  // a lane's slice of one Q2K row in one pass: EPL weights
+    static constexpr int NQ = EPL >= 16 ? EPL / 16 : 1;
+    uint32_t qs[NQ];  // 2-bit codes, one byte per 4 weights (word = 16 weights = one sub-block)
+    uint32_t sc;      // sub-block bytes: low nibble scale, high nibble min
+    uint32_t dm;      // block d | dmin << 16 (fp16)
+};
+
+// e0: first weight of the slice within the row (a multiple of EPL)
+template <int EPL>
+__device__ __forceinline__ void qk_rp_load(QkRp<EPL> &R, const uint8_t *W, const Planes &P, size_t row, int nblkf,
+                                           int e0) {
+    const uint8_t *qp = W + P.off[0] + row * size_t(nblkf) * 64 + e0 / 4;
+    const uint8_t *sp = W + P.off[1] + row * size_t(nblkf) * 16 + e0 / 16;
+    if constexpr (EPL == 64) {
+        const uint4 a = ldg_nc_v4(qp);
+        R.qs[0] = a.x; R.qs[1] = a.y; R.qs[2] = a.z; R.qs[3] = a.w;
+        R.sc = ldg_nc_u32(sp);
+    } else if constexpr (EPL == 32) {
+        const uint2 a = ldg_nc_v2(qp);
+        R.qs[0] = a.x; R.qs[1] = a.y;
+        R.sc = ldg_nc_u16(sp);
+    } else if constexpr (EPL == 16) {
+        R.qs[0] = ldg_nc_u32(qp);
+        R.sc = ldg_nc_u8(sp);
+    } else {
+        R.qs[0] = ldg_nc_u16(qp);
+        R.sc = ldg_nc_u8(sp);
+    }
+    R.dm = ldg_nc_u32(W + P.off[2] + (row * size_t(nblkf) + e0 / 256) * 4);
+}
+
+// sum over the slice of w_i * hh_i with w = d * sc * q - dmin * m per sub-block of 16:
+// d * sum_sb sc * (q . hh) - dmin * sum_sb m * (sum hh); hh = the lane's staged h (fp16 pairs), hs8 = sums of 8
+template <int EPL>
+__device__ __forceinline__ float qk_rp_dot(const QkRp<EPL> &R, const uint32_t (&hh)[EPL / 2],
+                                           const float (&hs8)[EPL / 8], uint32_t lane_tbl) {
+    constexpr int NSB = EPL >= 16 ? EPL / 16 : 1, NB = EPL >= 16 ? 4 : 2;  // sub-blocks, code bytes per sub-block
+    float A = 0.f, B = 0.f;
+#pragma unroll
+    for (int sb = 0; sb < NSB; sb++) {
+        __half2 a = __float2half2_rn(0.f), b = a;
+#pragma unroll
+        for (int bb = 0; bb < NB; bb++) {
+            const uint2 t = lds64(__byte_perm(R.qs[sb], lane_tbl, 0x7604 | (bb << 4)));
+            a = __hfma2(u32_as_half2(t.x), u32_as_half2(hh[sb * 8 + 2 * bb]), a);
+            b = __hfma2(u32_as_half2(t.y), u32_as_half2(hh[sb * 8 + 2 * bb + 1]), b);
+        }
+        const float2 s = __half22float2(__hadd2(a, b));
+        const uint32_t scb = (R.sc >> (8 * sb)) & 0xFFu;
+        const float hsum = EPL >= 16 ? hs8[2 * sb] + hs8[2 * sb + 1] : hs8[0];
+        A = fmaf(float(scb & 15u), s.x + s.y, A);
+        B = fmaf(float(scb >> 4), hsum, B);
+    }
+    const float dd = half_bits_to_float(uint16_t(R.dm & 0xFFFF));
+    const float dmin = half_bits_to_float(uint16_t(R.dm >> 16));
+    return dd * A - dmin * B;
+}
+
+template <int EPL>
+__global__ void __launch_bounds__(DD_THREADS, 1)
+    decode_down_kernel(const ExpertsDev ex, const float *__restrict__ h, const float *__restrict__ hs_in,
+                       const int32_t *__restrict__ ids, const float *__restrict__ wts, int k,
+                       float *__restrict__ out) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int d = ex.d, f = ex.f, fs = ex.fs;
+    const int nblkf = f / QK;
+    const int npass = f / (32 * EPL);
+    const uint32_t sbase = smem_u32(smem);
+    uint8_t *tb = smem + (DD_TABLE_ABS - sbase);
+    const DownSmemLayout L = dd_layout(k, f, fs);
+    __half *hq = reinterpret_cast<__half *>(tb + L.hq);
+    float *hsum = reinterpret_cast<float *>(tb + L.hsum);
+    float *hsl = reinterpret_cast<float *>(tb + L.hs);
+    float *wsc = reinterpret_cast<float *>(tb + L.wsc);
+    int *eid = reinterpret_cast<int *>(tb + L.eid);
+    const int n_units = d / DD_ROWS;
+    const int nW = gridDim.x * DD_WARPS;
+    const int u_first = warp * gridDim.x + blockIdx.x;
+    // the shared expert's rows of this warp's first unit go to L2 while the table is built
+    if (fs > 0 && u_first < n_units && lane == 0)
+        prefetch_l2(ex.sh_down + size_t(u_first) * DD_ROWS * fs, uint32_t(DD_ROWS * fs * 2));
+
+    // byte -> 4 fp16 table: entry b holds q_i = (b >> 2i) & 3, lane slot s at DD_TABLE_ABS + b * 256 + s * 8
+    for (int i = tid; i < 256 * 32; i += DD_THREADS) {
+        const int b = i >> 5;
+        const __half2 lo = __floats2half2_rn(float(b & 3), float((b >> 2) & 3));
+        const __half2 hi = __floats2half2_rn(float((b >> 4) & 3), float((b >> 6) & 3));
+        *reinterpret_cast<uint2 *>(tb + b * 256 + (i & 31) * 8) = make_uint2(half2_as_u32(lo), half2_as_u32(hi));
+    }
+
+    pdl_wait();  // h and hs come from the gate/up kernel, ids and weights from the router
+    // stage h_j (one warp per expert): fp16 of h * 2^e_j with max |h_j| * 2^e_j in [32, 64), and the fp32 sums of
+    // every 8 staged values
+    for (int j = warp; j < k; j += DD_WARPS) {
+        const float4 *hj = reinterpret_cast<const float4 *>(h + size_t(j) * f);
+        float m = 0.f;
+        for (int c = lane; c < f / 4; c += 32) {
+            const float4 v = hj[c];
+            m = fmaxf(m, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+        }
+        const int e = pow2_exponent_for(warp_max(m), 6);
+        const float sc = ldexpf(1.f, e);
+        for (int c = lane; c < f / 4; c += 32) {  // weights 4c .. 4c+3; f / 4 is a multiple of 32
+            const float4 v = hj[c];
+            const __half2 p0 = __floats2half2_rn(v.x * sc, v.y * sc), p1 = __floats2half2_rn(v.z * sc, v.w * sc);
+            *reinterpret_cast<uint2 *>(hq + size_t(j) * f + swz16(c / 2) * 8 + (c & 1) * 4) =
+                make_uint2(half2_as_u32(p0), half2_as_u32(p1));
+            const float2 a = __half22float2(p0), b = __half22float2(p1);
+            float s = (a.x + a.y) + (b.x + b.y);
+            s += __shfl_xor_sync(0xffffffffu, s, 1);
+            const int q = c / 2;  // index of the sum of weights 8q .. 8q+7
+            if ((lane & 1) == 0) hsum[j * (f / 8) + swz16(q / 4) * 4 + (q & 3)] = s;
+        }
+        if (lane == 0) {
+            wsc[j] = wts[j] * ldexpf(1.f, -e);
+            const int id = ids[j];
+            eid[j] = id;
+            if (id < 0 || id >= ex.E) set_device_error(DS4MOE_EDEVICE);
+        }
+    }
+    for (int i = tid * 4; i < fs; i += DD_THREADS * 4)
+        reinterpret_cast<float4 *>(hsl)[swz16(i / 4)] = *reinterpret_cast<const float4 *>(hs_in + i);
+    __syncthreads();
+
+    const uint32_t lane_tbl = DD_TABLE_ABS | uint32_t(lane * 8);
+    const int NS = npass * k;        // routed steps: (pass p, expert j) at n = p * k + j, two rows each
+    const int nsp = fs / 256;        // shared passes: lane slice 8 weights of [256 p, 256 p + 256)
+    for (int u = u_first; u < n_units; u += nW) {
+        const size_t r0 = size_t(u) * DD_ROWS;
+        // shared-expert ring (4 passes x 2 rows), primed first: these loads need nothing from the staging
+        uint4 sr[4][2];
+        auto sptr = [&](int p, int rr) { return ex.sh_down + (r0 + rr) * fs + p * 256 + lane * 8; };
+#pragma unroll
+        for (int s = 0; s < 4; s++)
+            if (s < nsp) {
+                sr[s][0] = ldg_nc_v4(sptr(s, 0));
+                sr[s][1] = ldg_nc_v4(sptr(s, 1));
+            }
+        if (u + nW < n_units && fs > 0 && lane == 0)
+            prefetch_l2(ex.sh_down + (r0 + size_t(nW) * DD_ROWS) * fs, uint32_t(DD_ROWS * fs * 2));
+        // routed ring: two steps in flight, both rows
+        auto rload = [&](QkRp<EPL> &R, int n, int rr) {
+            const int p = n / k, j = n - p * k;
+            const int e = eid[j];
+            if (e >= 0 && e < ex.E)
+                qk_rp_load<EPL>(R, ex.down + size_t(e) * ex.down_stride, ex.pd, r0 + rr, nblkf,
+                                p * 32 * EPL + lane * EPL);
+        };
+        QkRp<EPL> rg[2][2];
+#pragma unroll
+        for (int s = 0; s < 2; s++)
+            if (s < NS) {
+                rload(rg[s][0], s, 0);
+                rload(rg[s][1], s, 1);
+            }
+        float acc0 = 0.f, acc1 = 0.f;
+        for (int n0 = 0; n0 < NS; n0 += 2) {
+#pragma unroll
+            for (int s = 0; s < 2; s++) {
+                const int n = n0 + s;
+                if (n < NS) {
+                    const int p = n / k, j = n - p * k;
+                    const int e0 = p * 32 * EPL + lane * EPL;
+                    uint32_t hh[EPL / 2];
+                    float hs8[EPL / 8];
+                    const uint4 *hp = reinterpret_cast<const uint4 *>(hq + size_t(j) * f);
+                    const float *sp = hsum + j * (f / 8);
+#pragma unroll
+                    for (int i = 0; i < EPL / 8; i++) {
+                        const uint4 v = hp[swz16(e0 / 8 + i)];
+                        hh[4 * i] = v.x; hh[4 * i + 1] = v.y; hh[4 * i + 2] = v.z; hh[4 * i + 3] = v.w;
+                        const int q = e0 / 8 + i;
+                        hs8[i] = sp[swz16(q / 4) * 4 + (q & 3)];
+                    }
+                    const int e = eid[j];
+                    if (e >= 0 && e < ex.E) {
+                        acc0 = fmaf(wsc[j], qk_rp_dot<EPL>(rg[s][0], hh, hs8, lane_tbl), acc0);
+                        acc1 = fmaf(wsc[j], qk_rp_dot<EPL>(rg[s][1], hh, hs8, lane_tbl), acc1);
+                    }
+                    if (n + 2 < NS) {
+                        rload(rg[s][0], n + 2, 0);
+                        rload(rg[s][1], n + 2, 1);
+                    }
+                }
+            }
+        }
+        // shared expert
+        float as0 = 0.f, as1 = 0.f;
+        for (int p0 = 0; p0 < nsp; p0 += 4) {
+#pragma unroll
+            for (int s = 0; s < 4; s++) {
+                const int p = p0 + s;
+                if (p < nsp) {
+                    const float4 xa = reinterpret_cast<const float4 *>(hsl)[swz16(p * 64 + 2 * lane)];
+                    const float4 xb = reinterpret_cast<const float4 *>(hsl)[swz16(p * 64 + 2 * lane + 1)];
+                    as0 += bf16x8_dot(sr[s][0], xa, xb);
+                    as1 += bf16x8_dot(sr[s][1], xa, xb);
+                    if (p + 4 < nsp) {
+                        sr[s][0] = ldg_nc_v4(sptr(p + 4, 0));
+                        sr[s][1] = ldg_nc_v4(sptr(p + 4, 1));
+                    }
+                }
+            }
+        }
+        acc0 += as0;
+        acc1 += as1;
+        // reduce: lanes 0..15 end with row 0, lanes 16..31 with row 1
+        const bool hi = lane & 16;
+        float v = (hi ? acc1 : acc0) + __shfl_xor_sync(0xffffffffu, hi ? acc0 : acc1, 16);
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if ((lane & 15) == 0) out[r0 + (lane >> 4)] = v;
+    }
+}
+
+}  // namespace ds4

@@ -6,8 +6,7 @@
 #include <stdlib.h>
 
 #include "common.cuh"
-#include "decode.cuh"
-#include "decode_ring.cuh"
+#include "decode_gemv.cuh"
 #include "grouped_mma.cuh"
 #include "grouped_tc.cuh"
 #include "permute.cuh"
@@ -136,41 +135,22 @@ ExpertsDev to_dev(const ds4moe_experts *ex) {
 
 // ---- workspace layouts -----------------------------------------------------------------------------
 
+// The single-token GEMV kernels cover IQ2X gate/up with Q2K down, d <= 8192, and a down-kernel staging area
+// that fits in shared memory; everything else runs the grouped path with one token.
 bool decode_gemv_supported(const ds4moe_experts *ex, int k) {
-    const int vpl = ex->d / QK, wpl = ex->f / 512;
-    const bool vpl_ok = vpl == 1 || vpl == 2 || vpl == 4 || vpl == 8 || vpl == 16;
-    const bool wpl_ok = ex->f == 256 || wpl == 1 || wpl == 2 || wpl == 4 || wpl == 8;
-    return ex->fmt_gate == DS4MOE_FMT_IQ2X && ex->fmt_down == DS4MOE_FMT_Q2K && vpl_ok && wpl_ok && k <= 32;
+    if (ex->fmt_gate != DS4MOE_FMT_IQ2X || ex->fmt_down != DS4MOE_FMT_Q2K || k > 32) return false;
+    if (!dg_supported_d(ex->d) || !dd_supported_f(ex->f)) return false;
+    return dd_layout(k, ex->f, ex->f_shared).total <= 200 * 1024;
 }
 
 struct DecodeWs {
-    uint64_t h, sh_part, total;
-    int nch;
+    uint64_t h, hs, total;  // h_j = silu(G_j x) * (U_j x) for the k experts [k x f]; shared expert's h [f_shared]
 };
-// The ring-pipelined decode kernels cover d in {2048, 4096} (gate/up) and f = 2048 with f_shared a multiple of
-// 512 (down); other shapes run the register-batched kernels.
-// DS4MOE_DECODE=regs selects the register-batched kernels everywhere (A/B measurement).
-bool decode_regs_forced() {
-    static int v = -1;
-    if (v < 0) {
-        const char *e = getenv("DS4MOE_DECODE");
-        v = (e && e[0] == 'r' && e[1] == 'e') ? 1 : 0;
-    }
-    return v == 1;
-}
-bool gateup_ring(const ds4moe_experts *ex) { return !decode_regs_forced() && (ex->d == 4096 || ex->d == 2048); }
-bool down_ring(const ds4moe_experts *ex) {
-    return !decode_regs_forced() && ex->f == 2048 && ex->f_shared % 512 == 0 && ex->d <= 8192;
-}
-
 DecodeWs decode_ws(const ds4moe_experts *ex, int k) {
     DecodeWs w;
-    const int vpl = ex->d / QK;
-    const int ncv = vpl < 4 ? vpl : 4;
-    w.nch = gateup_ring(ex) ? ex->d / 512 : vpl / ncv;  // shared-expert partial-sum chunks per row
     w.h = 0;
-    w.sh_part = a256(uint64_t(k) * ex->f * 4);
-    w.total = w.sh_part + a256(uint64_t(w.nch) * 2 * (ex->f_shared > 0 ? ex->f_shared : 1) * 4);
+    w.hs = a256(uint64_t(k) * ex->f * 4);
+    w.total = w.hs + a256(uint64_t(ex->f_shared > 0 ? ex->f_shared : 1) * 4);
     return w;
 }
 
@@ -535,38 +515,15 @@ ds4moe_status ds4moe_decode_gateup(const ds4moe_experts *ex, const void *x_bf16,
     uint8_t *w8 = static_cast<uint8_t *>(ws);
     const ExpertsDev D = to_dev(ex);
     float *h = reinterpret_cast<float *>(w8 + W.h);
-    float *shp = reinterpret_cast<float *>(w8 + W.sh_part);
+    float *hs = reinterpret_cast<float *>(w8 + W.hs);
     const __nv_bfloat16 *x = static_cast<const __nv_bfloat16 *>(x_bf16);
-    const int grid = num_sms();
-    cudaStream_t st = cs(stream);
-    cudaError_t err;
-    if (gateup_ring(ex)) {
-        if (ex->d == 4096) {
-            if (!set_smem(decode_gateup_ring_kernel<16>, GR_DYN)) return DS4MOE_ECUDA;
-            err = launch_pdl(decode_gateup_ring_kernel<16>, dim3(grid), dim3(GR_THREADS), size_t(GR_DYN), st, D, x, ids,
-                             k, h, shp);
-        } else {
-            if (!set_smem(decode_gateup_ring_kernel<8>, GR_DYN)) return DS4MOE_ECUDA;
-            err = launch_pdl(decode_gateup_ring_kernel<8>, dim3(grid), dim3(GR_THREADS), size_t(GR_DYN), st, D, x, ids,
-                             k, h, shp);
-        }
-        if (err != cudaSuccess) {
-            (void)cudaGetLastError();
-            return DS4MOE_ECUDA;
-        }
-        return DS4MOE_OK;
-    }
-    switch (ex->d / QK) {
-#define GU_CASE(V)                                                                                              \
-    case V:                                                                                                     \
-        if (!set_smem(decode_gateup_iq2x_kernel<V>, gu_smem_bytes(ex->d))) return DS4MOE_ECUDA;                 \
-        err = launch_pdl(decode_gateup_iq2x_kernel<V>, dim3(grid), dim3(GU_THREADS), size_t(gu_smem_bytes(ex->d)), \
-                         st, D, x, ids, k, h, shp);                                                             \
-        break;
-        GU_CASE(1) GU_CASE(2) GU_CASE(4) GU_CASE(8) GU_CASE(16)
-#undef GU_CASE
-    default: return DS4MOE_EUNSUPPORTED;
-    }
+    const int smem = dg_smem_bytes(ex->d);
+    const int vpp = ex->d / QK < 8 ? ex->d / QK : 8;  // 8-vectors of a row per lane and pass
+    auto kern = vpp == 8 ? decode_gateup_kernel<8> : vpp == 4 ? decode_gateup_kernel<4>
+              : vpp == 2 ? decode_gateup_kernel<2> : decode_gateup_kernel<1>;
+    if (!set_smem(kern, smem)) return DS4MOE_ECUDA;
+    const cudaError_t err =
+        launch_pdl(kern, dim3(num_sms()), dim3(DG_THREADS), size_t(smem), cs(stream), D, x, ids, k, h, hs);
     if (err != cudaSuccess) {
         (void)cudaGetLastError();
         return DS4MOE_ECUDA;
@@ -587,34 +544,14 @@ ds4moe_status ds4moe_decode_down(const ds4moe_experts *ex, const int32_t *ids, c
     uint8_t *w8 = static_cast<uint8_t *>(ws);
     const ExpertsDev D = to_dev(ex);
     const float *h = reinterpret_cast<const float *>(w8 + W.h);
-    const float *shp = reinterpret_cast<const float *>(w8 + W.sh_part);
-    const int grid = num_sms();
-    const int wpl = ex->f <= 512 ? 1 : ex->f / 512;
-    const DownSmem L = down_smem_layout(k, wpl, ex->f_shared);
-    cudaStream_t st = cs(stream);
-    cudaError_t err;
-    if (down_ring(ex)) {
-        const DownRingSmem RL = down_ring_layout(k, ex->f_shared);
-        if (!set_smem(decode_down_ring_kernel, RL.total)) return DS4MOE_ECUDA;
-        err = launch_pdl(decode_down_ring_kernel, dim3(grid), dim3(DR_THREADS), size_t(RL.total), st, D, h, shp, W.nch,
-                         ids, weights, k, out);
-        if (err != cudaSuccess) {
-            (void)cudaGetLastError();
-            return DS4MOE_ECUDA;
-        }
-        return DS4MOE_OK;
-    }
-    switch (wpl) {
-#define DN_CASE(V)                                                                                               \
-    case V:                                                                                                      \
-        if (!set_smem(decode_down_q2k_kernel<V>, L.total)) return DS4MOE_ECUDA;                                  \
-        err = launch_pdl(decode_down_q2k_kernel<V>, dim3(grid), dim3(DN_THREADS), size_t(L.total), st, D, h, shp, \
-                         W.nch, ids, weights, k, out);                                                          \
-        break;
-        DN_CASE(1) DN_CASE(2) DN_CASE(4) DN_CASE(8)
-#undef DN_CASE
-    default: return DS4MOE_EUNSUPPORTED;
-    }
+    const float *hs = reinterpret_cast<const float *>(w8 + W.hs);
+    const int smem = dd_layout(k, ex->f, ex->f_shared).total;
+    const int epl = ex->f / 32 < 64 ? ex->f / 32 : 64;  // weights of a row per lane and pass
+    auto kern = epl == 64 ? decode_down_kernel<64> : epl == 32 ? decode_down_kernel<32>
+              : epl == 16 ? decode_down_kernel<16> : decode_down_kernel<8>;
+    if (!set_smem(kern, smem)) return DS4MOE_ECUDA;
+    const cudaError_t err = launch_pdl(kern, dim3(num_sms()), dim3(DD_THREADS), size_t(smem), cs(stream), D, h, hs,
+                                       ids, weights, k, out);
     if (err != cudaSuccess) {
         (void)cudaGetLastError();
         return DS4MOE_ECUDA;

@@ -154,24 +154,31 @@ ds4moe_status ds4moe_route(const void *x_bf16, int T, int d, const void *w_route
 size_t ds4moe_workspace_size(const ds4moe_experts *ex, int T, int k);
 
 /* Decode: out[B x d] (fp32) = the full layer output for B tokens, given the
- * routing (ids, weights) from ds4moe_route.  B = 1 runs the split-K GEMV
- * path (packed blocks streamed once, dequantized in registers, gate/up fused
- * with SwiGLU, down fused with the weighted combine and the shared expert);
- * B > 1 runs the grouped path internally (each touched expert read once). */
+ * routing (ids, weights) from ds4moe_route.  B = 1 runs the GEMV path (each
+ * selected expert's packed rows streamed once and dequantized on the fly,
+ * gate/up fused with SwiGLU, down fused with the weighted combine and the
+ * shared expert) when the layer is IQ2X gate/up with Q2K down, d <= 8192 and
+ * k <= 32; B > 1, and every other single-token layer, run the grouped path
+ * internally (each touched expert read once).  On the GEMV path x_bf16 is read
+ * before the wait on the preceding kernel (see ds4moe_decode_gateup), so x
+ * must not be written by the kernel launched just before this call on the
+ * same stream; ds4moe_route between the two satisfies this. */
 ds4moe_status ds4moe_expert_ffn_decode(const ds4moe_experts *ex, const void *x_bf16, int B, const int32_t *ids,
                                        const float *weights, int k, float *out, void *ws, size_t ws_bytes,
                                        ds4moe_stream stream);
 
-/* The two launches of ds4moe_expert_ffn_decode's single-token path, exposed
- * so a caller can place other work or timing events between them (B = 1;
- * gate/up IQ2X, down Q2K; d/256 in {1,2,4,8,16}; f in {256,...,4096} a power
- * of two times 256; same experts, workspace and stream for both).
- * ds4moe_decode_gateup streams the k selected experts' gate/up rows and the
- * shared expert's gate/up rows and leaves h_j = silu(G x) * (U x) and the
- * shared expert's partial sums in the workspace; ds4moe_decode_down reads
- * them and writes out[d] = sum_j w_j D_j h_j + Ds hs (fp32).  Both are
- * launched with programmatic dependent launch, so the shared-expert half of
- * the gate/up kernel overlaps the tail of the preceding router. */
+/* The two launches of ds4moe_expert_ffn_decode's single-token GEMV path,
+ * exposed so a caller can place other work or timing events between them
+ * (B = 1; same layer limits as that path; same experts, workspace and stream
+ * for both).  ds4moe_decode_gateup streams the k selected experts' gate/up
+ * rows and the shared expert's gate/up rows and leaves h_j = silu(G_j x) *
+ * (U_j x) (fp32, k x f) and the shared expert's hs (fp32, f_shared) at the
+ * start of the workspace; ds4moe_decode_down reads them and writes
+ * out[d] = sum_j w_j D_j h_j + Ds hs (fp32).  Both are launched with
+ * programmatic dependent launch: the gate/up kernel reads x and streams the
+ * shared expert before it waits for the preceding kernel (normally the
+ * router's top-k, which produces ids), so x must be complete before that
+ * kernel starts; the down kernel reads nothing before its wait. */
 ds4moe_status ds4moe_decode_gateup(const ds4moe_experts *ex, const void *x_bf16, const int32_t *ids, int k, void *ws,
                                    size_t ws_bytes, ds4moe_stream stream);
 ds4moe_status ds4moe_decode_down(const ds4moe_experts *ex, const int32_t *ids, const float *weights, int k,
@@ -182,11 +189,13 @@ ds4moe_status ds4moe_decode_down(const ds4moe_experts *ex, const int32_t *ids, c
  * of HBM and forbids further allocation, or a plugin host that exposes no
  * allocator.  The paper has no counterpart: this is a library convenience.
  * Same computation and arguments as ds4moe_expert_ffn_decode with B = 1 (and
- * the same format limits as ds4moe_decode_gateup), but the scratch comes from
+ * the same layer limits as ds4moe_decode_gateup), but the scratch comes from
  * a 1 MiB array compiled into the library, which every GPU that loads the
- * library holds until the process exits.  Layers whose decode scratch
- * (4 * (k*f + 2*f_shared*ceil(d/1024)) bytes, rounded) exceeds 1 MiB are
- * rejected with DS4MOE_ENOWORKSPACE.  Nothing is allocated: no cudaMalloc, no
+ * library holds until the process exits.  Layers outside the GEMV path's
+ * limits are rejected with DS4MOE_EUNSUPPORTED, and a layer whose decode
+ * scratch (4 * (k*f + f_shared) bytes, each part rounded up to 256) exceeds
+ * 1 MiB with DS4MOE_ENOWORKSPACE (under the present limits every supported
+ * layer fits).  Nothing is allocated: no cudaMalloc, no
  * cudaFree.  The first call on a device looks up the array's device address
  * (once per device, with that device current); make that first call before
  * any stream capture.  All calls share the one array, which keeps the last

@@ -45,10 +45,11 @@ def test_noalloc_matches_workspace_entry_two_calls(ds4, shape):
         parity.assert_output_close(got.double().cpu().numpy(), ref.double().cpu().numpy(), "noalloc call %d" % t)
 
 
-def test_noalloc_rejects_layer_beyond_fixed_scratch(ds4):
-    # shared-expert partial sums alone need 4 * 2 * 65536 * 4 bytes = 2 MiB > 1 MiB: refused before any launch
+def test_noalloc_rejects_layer_beyond_its_limits(ds4):
+    # f_shared = 65536: the down kernel cannot stage the shared expert's h on chip, so the GEMV path (the only
+    # one the fixed scratch serves) does not take the layer; refused before any launch
     ex = ds4.Experts(4096, 2048, 256, 65536, 0, 0, 1, 1 << 20, 1 << 21, 1 << 22, 1 << 24, 1 << 24, 1 << 24, 1 << 23,
                      1 << 25, 1 << 26, 1 << 27)
     fake = ctypes.c_void_p(1 << 20)
     rc = ds4.lib().ds4moe_expert_ffn_decode_noalloc(ctypes.byref(ex), fake, fake, fake, 8, fake, None)
-    assert rc == 4  # DS4MOE_ENOWORKSPACE
+    assert rc == 2  # DS4MOE_EUNSUPPORTED
