@@ -81,30 +81,23 @@ __device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes) {
 // conflict within a quarter-warp.
 __host__ __device__ __forceinline__ int swz16(int c) { return c ^ ((c >> 3) & 7); }
 
-// Butterfly reduce-scatter over the 32 lanes of 16 per-lane partial sums: afterwards lanes 2v and 2v+1 both
-// hold the full sum of value v = (lane >> 1) & 15.
-__device__ __forceinline__ float reduce16(float (&v)[16], int lane) {
+// Butterfly reduce-scatter over the 32 lanes of N per-lane partial sums (N a power of two <= 16): afterwards the
+// 32 / N lanes lane = v * (32 / N) + i (i < 32 / N) all hold the full sum of value v.
+template <int N>
+__device__ __forceinline__ float reduce_scatter(float (&v)[N], int lane) {
 #pragma unroll
-    for (int i = 0; i < 8; i++) {
-        const bool hi = lane & 16;
-        const float send = hi ? v[i] : v[i + 8], keep = hi ? v[i + 8] : v[i];
-        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
-    }
+    for (int n = N / 2, o = 16; n >= 1; n >>= 1, o >>= 1) {
+        const bool hi = lane & o;
 #pragma unroll
-    for (int i = 0; i < 4; i++) {
-        const bool hi = lane & 8;
-        const float send = hi ? v[i] : v[i + 4], keep = hi ? v[i + 4] : v[i];
-        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+        for (int i = 0; i < n; i++) {
+            const float send = hi ? v[i] : v[i + n], keep = hi ? v[i + n] : v[i];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
     }
+    float r = v[0];
 #pragma unroll
-    for (int i = 0; i < 2; i++) {
-        const bool hi = lane & 4;
-        const float send = hi ? v[i] : v[i + 2], keep = hi ? v[i + 2] : v[i];
-        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
-    }
-    const bool hi = lane & 2;
-    float r = (hi ? v[1] : v[0]) + __shfl_xor_sync(0xffffffffu, hi ? v[0] : v[1], 2);
-    return r + __shfl_xor_sync(0xffffffffu, r, 1);
+    for (int o = 16 / N; o >= 1; o >>= 1) r += __shfl_xor_sync(0xffffffffu, r, o);
+    return r;
 }
 
 // ============================================================================ gate / up
@@ -112,8 +105,9 @@ __device__ __forceinline__ float reduce16(float (&v)[16], int lane) {
 constexpr int DG_WARPS = 16;
 constexpr int DG_THREADS = DG_WARPS * 32;
 constexpr uint32_t DG_TABLE_ABS = 0x10000;  // absolute shared address of the 64 KB codebook table
-constexpr int DG_ROWS = 8;                  // gate/up row pairs per unit (routed and shared)
+constexpr int DG_ROWS = 4;                  // gate/up row pairs per unit (routed and shared): 4 or 8
 constexpr int DG_MAX_D = 8192;
+constexpr int DG_RING = 4;                  // row slices whose packed data is in flight per lane (divides 2 DG_ROWS)
 
 // Contraction lengths the gate/up kernel takes: d = 256 * nblk with nblk in {1, 2, 4, 8, 16, 32}.  A lane owns
 // VPP = min(nblk, 8) consecutive 8-vectors of a row per pass; nblk / VPP passes.
@@ -195,9 +189,9 @@ __device__ __forceinline__ float bf16x8_dot(const uint4 w, const float4 a, const
     return s;
 }
 
-// Units: shared-expert units first (rows 8u .. 8u+7 of Gs, Us), then routed units (expert slot j, rows
-// 8i .. 8i+7).  Row-matrix index rr = 2 * (row - first row) + (0 gate, 1 up).
-template <int VPP>
+// Units of NR row pairs: shared-expert units first (rows NR u .. NR u + NR - 1 of Gs, Us), then routed units
+// (expert slot j, rows NR i ..).  Row-matrix index rr = 2 * (row - first row) + (0 gate, 1 up).
+template <int VPP, int NR>
 __global__ void __launch_bounds__(DG_THREADS, 1)
     decode_gateup_kernel(const ExpertsDev ex, const __nv_bfloat16 *__restrict__ x, const int32_t *__restrict__ ids,
                          int k, float *__restrict__ h_out, float *__restrict__ hs_out) {
@@ -213,29 +207,32 @@ __global__ void __launch_bounds__(DG_THREADS, 1)
     float *x32 = reinterpret_cast<float *>(tbl + 65536 + d * 2);
     const uint32_t x16_s = DG_TABLE_ABS + 65536;
 
-    const int n_sh = fs / DG_ROWS;
-    const int upe = f / DG_ROWS;  // routed units per expert
+    constexpr int NRR = 2 * NR;      // row-matrices per unit
+    constexpr int LPV = 32 / NRR;    // lanes that hold one row-matrix sum after the reduce-scatter
+    const int n_sh = fs / NR;
+    const int upe = f / NR;  // routed units per expert
     const int n_all = n_sh + k * upe;
     const int nW = gridDim.x * DG_WARPS;
     const int u_first = warp * gridDim.x + blockIdx.x;
     // the shared expert's rows of this warp's first unit go to L2 while the tables are built
-    if (u_first < n_sh && lane < 2 * DG_ROWS)
-        prefetch_l2((lane & 1 ? ex.sh_up : ex.sh_gate) + size_t(u_first * DG_ROWS + (lane >> 1)) * d, uint32_t(d * 2));
+    if (u_first < n_sh && lane < NRR)
+        prefetch_l2((lane & 1 ? ex.sh_up : ex.sh_gate) + size_t(u_first * NR + (lane >> 1)) * d, uint32_t(d * 2));
 
     // prologue, one global round trip: every thread loads its codebook entry and its 8 activations together,
     // then writes the codebook table (entry e, lane slot s at DG_TABLE_ABS + e * 256 + s * 16: 8 grid values as
     // fp16), the fp32 activations, and after the block-wide max the fp16 activations scaled by the power of two
     // that puts max |x| in [32, 64)
-    const int e_cb = tid >> 1;
-    const uint2 raw = *reinterpret_cast<const uint2 *>(ex.codebook + e_cb * 8);
-    constexpr int XPT = DG_MAX_D / (DG_THREADS * 8);  // 8-element activation chunks per thread (at most)
+    static_assert(DG_THREADS >= 512, "two threads per codebook entry");
+    const int e_cb = tid >> 1;  // threads 0 .. 511 build the table
+    const uint2 raw = tid < 512 ? *reinterpret_cast<const uint2 *>(ex.codebook + e_cb * 8) : make_uint2(0, 0);
+    constexpr int XPT = (DG_MAX_D + DG_THREADS * 8 - 1) / (DG_THREADS * 8);  // 8-element chunks per thread
     uint4 xv[XPT];
 #pragma unroll
     for (int c = 0; c < XPT; c++) {
         const int i = (tid + c * DG_THREADS) * 8;
         if (i < d) xv[c] = *reinterpret_cast<const uint4 *>(x + i);
     }
-    {
+    if (tid < 512) {
         const uint32_t b[2] = {raw.x, raw.y};
         __half2 hv[4];
 #pragma unroll
@@ -283,16 +280,16 @@ __global__ void __launch_bounds__(DG_THREADS, 1)
     const uint32_t lane_tbl = DG_TABLE_ABS | uint32_t((lane & 15) * 16);
     bool waited = false;
     for (int u = u_first; u < n_all; u += nW) {
-        float acc[16];
+        float acc[NRR];
 #pragma unroll
-        for (int i = 0; i < 16; i++) acc[i] = 0.f;
+        for (int i = 0; i < NRR; i++) acc[i] = 0.f;
         if (u < n_sh) {
             // shared expert (bf16): pass p covers elements [256 p, 256 p + 256), lane slice 8 elements; ring of 8 rows
-            const size_t r0 = size_t(u) * DG_ROWS;
-            const int ns = d / 256, T = ns * 16;
+            const size_t r0 = size_t(u) * NR;
+            const int ns = d / 256, T = ns * NRR;
             auto wptr = [&](int t) {
-                const int rr = t & 15;
-                return (rr & 1 ? ex.sh_up : ex.sh_gate) + (r0 + (rr >> 1)) * d + (t >> 4) * 256 + lane * 8;
+                const int rr = t % NRR;
+                return (rr & 1 ? ex.sh_up : ex.sh_gate) + (r0 + (rr >> 1)) * d + (t / NRR) * 256 + lane * 8;
             };
             uint4 ring[8];
 #pragma unroll
@@ -301,15 +298,15 @@ __global__ void __launch_bounds__(DG_THREADS, 1)
                 const float4 xa = reinterpret_cast<const float4 *>(x32)[swz16(p * 64 + 2 * lane)];
                 const float4 xb = reinterpret_cast<const float4 *>(x32)[swz16(p * 64 + 2 * lane + 1)];
 #pragma unroll
-                for (int rr = 0; rr < 16; rr++) {
+                for (int rr = 0; rr < NRR; rr++) {
                     acc[rr] += bf16x8_dot(ring[rr & 7], xa, xb);
-                    const int tn = p * 16 + rr + 8;
+                    const int tn = p * NRR + rr + 8;
                     if (tn < T) ring[rr & 7] = ldg_nc_v4(wptr(tn));
                 }
             }
-            const float v = reduce16(acc, lane);
-            const float up = __shfl_xor_sync(0xffffffffu, v, 2);  // lanes 4i: gate of row i; 4i + 2: up
-            if ((lane & 3) == 0) hs_out[r0 + (lane >> 2)] = silu(v) * up;
+            const float v = reduce_scatter<NRR>(acc, lane);
+            const float up = __shfl_xor_sync(0xffffffffu, v, LPV);  // gate of row i on lane 2 i LPV, up next
+            if (lane % (2 * LPV) == 0) hs_out[r0 + lane / (2 * LPV)] = silu(v) * up;
             continue;
         }
         if (!waited) {
@@ -318,36 +315,37 @@ __global__ void __launch_bounds__(DG_THREADS, 1)
         }
         const int uu = u - n_sh;
         const int j = uu / upe;
-        const size_t r0 = size_t(uu % upe) * DG_ROWS;
+        const size_t r0 = size_t(uu % upe) * NR;
         const int e = ids[j];
         if (e < 0 || e >= ex.E) {
             if (lane == 0) set_device_error(DS4MOE_EDEVICE);
             continue;
         }
         const uint8_t *G = ex.gate + size_t(e) * ex.gate_stride, *U = ex.up + size_t(e) * ex.up_stride;
-        const int T = npass * 16;
+        const int T = npass * NRR;
         auto load = [&](IqRp<VPP> &R, int t) {
-            const int rr = t & 15;
-            iq_rp_load<VPP>(R, rr & 1 ? U : G, ex.pg, r0 + (rr >> 1), nblk, (t >> 4) * 32 * VPP + lane * VPP);
+            const int rr = t % NRR;
+            iq_rp_load<VPP>(R, rr & 1 ? U : G, ex.pg, r0 + (rr >> 1), nblk, (t / NRR) * 32 * VPP + lane * VPP);
         };
-        IqRp<VPP> ring[4];
+        IqRp<VPP> ring[DG_RING];
 #pragma unroll
-        for (int s = 0; s < 4; s++) load(ring[s], s);
+        for (int s = 0; s < DG_RING; s++) load(ring[s], s);
         for (int p = 0; p < npass; p++) {
             const int v0 = p * 32 * VPP + lane * VPP;
             uint4 xr[VPP];
 #pragma unroll
             for (int v = 0; v < VPP; v++) xr[v] = lds128(x16_s + swz16(v0 + v) * 16);
 #pragma unroll
-            for (int rr = 0; rr < 16; rr++) {
-                acc[rr] += iq_rp_dot<VPP>(ring[rr & 3], xr, v0, lane_tbl);
-                const int tn = p * 16 + rr + 4;
-                if (tn < T) load(ring[rr & 3], tn);
+            for (int rr = 0; rr < NRR; rr++) {
+                acc[rr] += iq_rp_dot<VPP>(ring[rr % DG_RING], xr, v0, lane_tbl);
+                const int tn = p * NRR + rr + DG_RING;
+                if (tn < T) load(ring[rr % DG_RING], tn);
             }
         }
-        const float v = reduce16(acc, lane);
-        const float up = __shfl_xor_sync(0xffffffffu, v, 2);
-        if ((lane & 3) == 0) h_out[size_t(j) * f + r0 + (lane >> 2)] = silu(v * inv_xs) * (up * inv_xs);
+        const float v = reduce_scatter<NRR>(acc, lane);
+        const float up = __shfl_xor_sync(0xffffffffu, v, LPV);
+        if (lane % (2 * LPV) == 0)
+            h_out[size_t(j) * f + r0 + lane / (2 * LPV)] = silu(v * inv_xs) * (up * inv_xs);
     }
 }
 

@@ -519,8 +519,8 @@ ds4moe_status ds4moe_decode_gateup(const ds4moe_experts *ex, const void *x_bf16,
     const __nv_bfloat16 *x = static_cast<const __nv_bfloat16 *>(x_bf16);
     const int smem = dg_smem_bytes(ex->d);
     const int vpp = ex->d / QK < 8 ? ex->d / QK : 8;  // 8-vectors of a row per lane and pass
-    auto kern = vpp == 8 ? decode_gateup_kernel<8> : vpp == 4 ? decode_gateup_kernel<4>
-              : vpp == 2 ? decode_gateup_kernel<2> : decode_gateup_kernel<1>;
+    auto kern = vpp == 8 ? decode_gateup_kernel<8, DG_ROWS> : vpp == 4 ? decode_gateup_kernel<4, DG_ROWS>
+              : vpp == 2 ? decode_gateup_kernel<2, DG_ROWS> : decode_gateup_kernel<1, DG_ROWS>;
     if (!set_smem(kern, smem)) return DS4MOE_ECUDA;
     const cudaError_t err =
         launch_pdl(kern, dim3(num_sms()), dim3(DG_THREADS), size_t(smem), cs(stream), D, x, ids, k, h, hs);
