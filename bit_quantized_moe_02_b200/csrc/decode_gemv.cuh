@@ -362,17 +362,27 @@ __host__ __device__ __forceinline__ bool dd_supported_f(int f) {
     const int nblk = f / QK;
     return f % QK == 0 && nblk >= 1 && nblk <= 32 && (nblk & (nblk - 1)) == 0;
 }
+__host__ __device__ __forceinline__ int dd_epl(int f) { return f / 32 < 64 ? f / 32 : 64; }
 
+// Staged h is stored per lane slice (the EPL weights one lane owns in one pass), each slice padded by 16 bytes
+// when that keeps the 8 lanes of a quarter-warp on distinct banks; the lane then reads its slice with
+// immediate offsets.  hq: fp16 h * 2^e_j, slice stride hq_sb; hsum: fp32 sums of 8 staged values, stride hs_sb.
 struct DownSmemLayout {
-    int hq, hsum, hs, wsc, eid, total;  // byte offsets from the table base; total = dynamic bytes to request
+    int hq, hq_sb, hq_eb, hsum, hs_sb, hs_eb, hs, wsc, eid, total;  // byte offsets from the table base / strides
 };
 __host__ __device__ __forceinline__ DownSmemLayout dd_layout(int k, int f, int fs) {
     DownSmemLayout L;
-    L.hq = 65536;                                   // k x f fp16: h_j * 2^e_j
-    L.hsum = L.hq + k * f * 2;                      // k x f/8 floats: sums of 8 consecutive staged values
-    L.hs = L.hsum + ((k * (f / 8) * 4 + 15) & ~15);  // fs floats: shared-expert h
-    L.wsc = L.hs + ((fs * 4 + 15) & ~15);           // k floats: w_j * 2^-e_j
-    L.eid = L.wsc + ((k * 4 + 15) & ~15);           // k ints: expert ids
+    const int epl = dd_epl(f);
+    const int nsl = f / epl;                           // lane slices per expert (32 per pass)
+    L.hq_sb = epl * 2 + (epl >= 16 ? 16 : 0);
+    L.hq_eb = nsl * L.hq_sb;
+    L.hs_sb = epl / 8 * 4 + (epl == 64 ? 16 : 0);
+    L.hs_eb = nsl * L.hs_sb;
+    L.hq = 65536;
+    L.hsum = L.hq + ((k * L.hq_eb + 15) & ~15);
+    L.hs = L.hsum + ((k * L.hs_eb + 15) & ~15);        // fs floats: shared-expert h (16-byte chunks swizzled)
+    L.wsc = L.hs + ((fs * 4 + 15) & ~15);              // k floats: w_j * 2^-e_j
+    L.eid = L.wsc + ((k * 4 + 15) & ~15);              // k ints: expert ids
     L.total = int(DD_TABLE_ABS) + L.eid + ((k * 4 + 15) & ~15);
     return L;
 }
@@ -385,7 +395,8 @@ struct QkRp {  // a lane's slice of one Q2K row in one pass: EPL weights
     uint32_t dm;      // block d | dmin << 16 (fp16)
 };
 
-// e0: first weight of the slice within the row (a multiple of EPL)
+// p: the row's bytes in the code plane at the slice (row * f / 4 + e0 / 4); the scale and d/dmin planes follow
+// from the same slice position
 template <int EPL>
 __device__ __forceinline__ void qk_rp_load(QkRp<EPL> &R, const uint8_t *W, const Planes &P, size_t row, int nblkf,
                                            int e0) {
@@ -436,6 +447,32 @@ __device__ __forceinline__ float qk_rp_dot(const QkRp<EPL> &R, const uint32_t (&
     return dd * A - dmin * B;
 }
 
+// the lane's staged slice (EPL fp16 and EPL / 8 sums) at shared addresses hq_addr, hs_addr
+template <int EPL>
+__device__ __forceinline__ void dd_slice_load(uint32_t hq_addr, uint32_t hs_addr, uint32_t (&hh)[EPL / 2],
+                                              float (&hs8)[EPL / 8]) {
+#pragma unroll
+    for (int i = 0; i < EPL / 8; i++) {
+        const uint4 v = lds128(hq_addr + 16 * i);
+        hh[4 * i] = v.x; hh[4 * i + 1] = v.y; hh[4 * i + 2] = v.z; hh[4 * i + 3] = v.w;
+    }
+    if constexpr (EPL >= 32) {
+#pragma unroll
+        for (int i = 0; i < EPL / 32; i++) {
+            const uint4 v = lds128(hs_addr + 16 * i);
+            hs8[4 * i] = __uint_as_float(v.x); hs8[4 * i + 1] = __uint_as_float(v.y);
+            hs8[4 * i + 2] = __uint_as_float(v.z); hs8[4 * i + 3] = __uint_as_float(v.w);
+        }
+    } else if constexpr (EPL == 16) {
+        const uint2 v = lds64(hs_addr);
+        hs8[0] = __uint_as_float(v.x); hs8[1] = __uint_as_float(v.y);
+    } else {
+        uint32_t v;
+        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(hs_addr));
+        hs8[0] = __uint_as_float(v);
+    }
+}
+
 template <int EPL>
 __global__ void __launch_bounds__(DD_THREADS, 1)
     decode_down_kernel(const ExpertsDev ex, const float *__restrict__ h, const float *__restrict__ hs_in,
@@ -449,8 +486,6 @@ __global__ void __launch_bounds__(DD_THREADS, 1)
     const uint32_t sbase = smem_u32(smem);
     uint8_t *tb = smem + (DD_TABLE_ABS - sbase);
     const DownSmemLayout L = dd_layout(k, f, fs);
-    __half *hq = reinterpret_cast<__half *>(tb + L.hq);
-    float *hsum = reinterpret_cast<float *>(tb + L.hsum);
     float *hsl = reinterpret_cast<float *>(tb + L.hs);
     float *wsc = reinterpret_cast<float *>(tb + L.wsc);
     int *eid = reinterpret_cast<int *>(tb + L.eid);
@@ -470,27 +505,79 @@ __global__ void __launch_bounds__(DD_THREADS, 1)
     }
 
     pdl_wait();  // h and hs come from the gate/up kernel, ids and weights from the router
+
+    const int NS = npass * k;  // routed steps: (pass p, expert slot j), both rows of the unit
+    const int nsp = fs / 256;  // shared passes: lane slice 8 weights of [256 p, 256 p + 256)
+    // Rings of the unit in progress: routed steps n and n + 1 (both rows), shared passes p .. p + 3 (both rows).
+    // (Filling the first unit's rings before the staging below was measured slower: those loads then compete
+    // with the staging's reads of h, which every warp waits for.)
+    QkRp<EPL> rg[2][2];
+    uint4 sr[4][2];
+    int pn = 0, jn = 0;  // next routed step to load
+    auto rload = [&](QkRp<EPL> &R, int e, size_t row, int p) {
+        if (e >= 0 && e < ex.E)
+            qk_rp_load<EPL>(R, ex.down + size_t(e) * ex.down_stride, ex.pd, row, nblkf, p * 32 * EPL + lane * EPL);
+    };
+    auto prime = [&](int u, const int *idv) {
+        const size_t r0 = size_t(u) * DD_ROWS;
+        pn = 0;
+        jn = 0;
+#pragma unroll
+        for (int s = 0; s < 2; s++)
+            if (s < NS) {
+                const int e = idv[jn];
+                rload(rg[s][0], e, r0, pn);
+                rload(rg[s][1], e, r0 + 1, pn);
+                if (++jn == k) { jn = 0; pn++; }
+            }
+        const __nv_bfloat16 *s0 = ex.sh_down + r0 * fs + lane * 8;
+#pragma unroll
+        for (int s = 0; s < 4; s++)
+            if (s < nsp) {
+                sr[s][0] = ldg_nc_v4(s0 + s * 256);
+                sr[s][1] = ldg_nc_v4(s0 + fs + s * 256);
+            }
+    };
+
     // stage h_j (one warp per expert): fp16 of h * 2^e_j with max |h_j| * 2^e_j in [32, 64), and the fp32 sums of
-    // every 8 staged values
+    // every 8 staged values, both in per-lane-slice order.  Loads go out 4 per lane at a time.
     for (int j = warp; j < k; j += DD_WARPS) {
         const float4 *hj = reinterpret_cast<const float4 *>(h + size_t(j) * f);
+        const int nc = f / 128;  // float4 chunks per lane (a multiple of 2)
         float m = 0.f;
-        for (int c = lane; c < f / 4; c += 32) {
-            const float4 v = hj[c];
-            m = fmaxf(m, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+        for (int c0 = 0; c0 < nc; c0 += 4) {
+            float4 v[4];
+#pragma unroll
+            for (int i = 0; i < 4; i++)
+                if (c0 + i < nc) v[i] = hj[(c0 + i) * 32 + lane];
+#pragma unroll
+            for (int i = 0; i < 4; i++)
+                if (c0 + i < nc)
+                    m = fmaxf(m, fmaxf(fmaxf(fabsf(v[i].x), fabsf(v[i].y)), fmaxf(fabsf(v[i].z), fabsf(v[i].w))));
         }
         const int e = pow2_exponent_for(warp_max(m), 6);
         const float sc = ldexpf(1.f, e);
-        for (int c = lane; c < f / 4; c += 32) {  // weights 4c .. 4c+3; f / 4 is a multiple of 32
-            const float4 v = hj[c];
-            const __half2 p0 = __floats2half2_rn(v.x * sc, v.y * sc), p1 = __floats2half2_rn(v.z * sc, v.w * sc);
-            *reinterpret_cast<uint2 *>(hq + size_t(j) * f + swz16(c / 2) * 8 + (c & 1) * 4) =
-                make_uint2(half2_as_u32(p0), half2_as_u32(p1));
-            const float2 a = __half22float2(p0), b = __half22float2(p1);
-            float s = (a.x + a.y) + (b.x + b.y);
-            s += __shfl_xor_sync(0xffffffffu, s, 1);
-            const int q = c / 2;  // index of the sum of weights 8q .. 8q+7
-            if ((lane & 1) == 0) hsum[j * (f / 8) + swz16(q / 4) * 4 + (q & 3)] = s;
+        for (int c0 = 0; c0 < nc; c0 += 4) {
+            float4 v[4];
+#pragma unroll
+            for (int i = 0; i < 4; i++)
+                if (c0 + i < nc) v[i] = hj[(c0 + i) * 32 + lane];
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                if (c0 + i < nc) {
+                    const int c = (c0 + i) * 32 + lane;  // weights 4c .. 4c+3
+                    const __half2 p0 = __floats2half2_rn(v[i].x * sc, v[i].y * sc);
+                    const __half2 p1 = __floats2half2_rn(v[i].z * sc, v[i].w * sc);
+                    const int el = 4 * c, slice = el / EPL, o = el % EPL;  // slice = pass * 32 + lane
+                    *reinterpret_cast<uint2 *>(tb + L.hq + j * L.hq_eb + slice * L.hq_sb + o * 2) =
+                        make_uint2(half2_as_u32(p0), half2_as_u32(p1));
+                    const float2 a = __half22float2(p0), b = __half22float2(p1);
+                    float s = (a.x + a.y) + (b.x + b.y);
+                    s += __shfl_xor_sync(0xffffffffu, s, 1);
+                    if ((lane & 1) == 0)
+                        *reinterpret_cast<float *>(tb + L.hsum + j * L.hs_eb + slice * L.hs_sb + (o / 8) * 4) = s;
+                }
+            }
         }
         if (lane == 0) {
             wsc[j] = wts[j] * ldexpf(1.f, -e);
@@ -504,87 +591,61 @@ __global__ void __launch_bounds__(DD_THREADS, 1)
     __syncthreads();
 
     const uint32_t lane_tbl = DD_TABLE_ABS | uint32_t(lane * 8);
-    const int NS = npass * k;        // routed steps: (pass p, expert j) at n = p * k + j, two rows each
-    const int nsp = fs / 256;        // shared passes: lane slice 8 weights of [256 p, 256 p + 256)
+    const uint32_t hq_lane = DD_TABLE_ABS + uint32_t(L.hq + lane * L.hq_sb);
+    const uint32_t hs_lane = DD_TABLE_ABS + uint32_t(L.hsum + lane * L.hs_sb);
     for (int u = u_first; u < n_units; u += nW) {
         const size_t r0 = size_t(u) * DD_ROWS;
-        // shared-expert ring (4 passes x 2 rows), primed first: these loads need nothing from the staging
-        uint4 sr[4][2];
-        auto sptr = [&](int p, int rr) { return ex.sh_down + (r0 + rr) * fs + p * 256 + lane * 8; };
-#pragma unroll
-        for (int s = 0; s < 4; s++)
-            if (s < nsp) {
-                sr[s][0] = ldg_nc_v4(sptr(s, 0));
-                sr[s][1] = ldg_nc_v4(sptr(s, 1));
-            }
+        prime(u, eid);
         if (u + nW < n_units && fs > 0 && lane == 0)
             prefetch_l2(ex.sh_down + (r0 + size_t(nW) * DD_ROWS) * fs, uint32_t(DD_ROWS * fs * 2));
-        // routed ring: two steps in flight, both rows
-        auto rload = [&](QkRp<EPL> &R, int n, int rr) {
-            const int p = n / k, j = n - p * k;
-            const int e = eid[j];
-            if (e >= 0 && e < ex.E)
-                qk_rp_load<EPL>(R, ex.down + size_t(e) * ex.down_stride, ex.pd, r0 + rr, nblkf,
-                                p * 32 * EPL + lane * EPL);
-        };
-        QkRp<EPL> rg[2][2];
-#pragma unroll
-        for (int s = 0; s < 2; s++)
-            if (s < NS) {
-                rload(rg[s][0], s, 0);
-                rload(rg[s][1], s, 1);
-            }
+        // shared expert first (bf16 rows, fp32 hs): it covers the latency of the routed ring's first loads
         float acc0 = 0.f, acc1 = 0.f;
+        if (nsp > 0) {
+            const __nv_bfloat16 *s0 = ex.sh_down + r0 * fs + lane * 8, *s1 = s0 + fs;
+            for (int p0 = 0; p0 < nsp; p0 += 4) {
+#pragma unroll
+                for (int s = 0; s < 4; s++) {
+                    const int p = p0 + s;
+                    if (p < nsp) {
+                        const float4 xa = reinterpret_cast<const float4 *>(hsl)[swz16(p * 64 + 2 * lane)];
+                        const float4 xb = reinterpret_cast<const float4 *>(hsl)[swz16(p * 64 + 2 * lane + 1)];
+                        acc0 += bf16x8_dot(sr[s][0], xa, xb);
+                        acc1 += bf16x8_dot(sr[s][1], xa, xb);
+                        if (p + 4 < nsp) {
+                            sr[s][0] = ldg_nc_v4(s0 + (p + 4) * 256);
+                            sr[s][1] = ldg_nc_v4(s1 + (p + 4) * 256);
+                        }
+                    }
+                }
+            }
+        }
+        // routed experts
+        int p = 0, j = 0;  // step being consumed
         for (int n0 = 0; n0 < NS; n0 += 2) {
 #pragma unroll
             for (int s = 0; s < 2; s++) {
-                const int n = n0 + s;
-                if (n < NS) {
-                    const int p = n / k, j = n - p * k;
-                    const int e0 = p * 32 * EPL + lane * EPL;
+                if (n0 + s < NS) {
                     uint32_t hh[EPL / 2];
                     float hs8[EPL / 8];
-                    const uint4 *hp = reinterpret_cast<const uint4 *>(hq + size_t(j) * f);
-                    const float *sp = hsum + j * (f / 8);
-#pragma unroll
-                    for (int i = 0; i < EPL / 8; i++) {
-                        const uint4 v = hp[swz16(e0 / 8 + i)];
-                        hh[4 * i] = v.x; hh[4 * i + 1] = v.y; hh[4 * i + 2] = v.z; hh[4 * i + 3] = v.w;
-                        const int q = e0 / 8 + i;
-                        hs8[i] = sp[swz16(q / 4) * 4 + (q & 3)];
-                    }
+                    const int sl = p * 32;  // slice offset of this pass
+                    dd_slice_load<EPL>(hq_lane + j * L.hq_eb + sl * L.hq_sb, hs_lane + j * L.hs_eb + sl * L.hs_sb, hh,
+                                       hs8);
                     const int e = eid[j];
                     if (e >= 0 && e < ex.E) {
-                        acc0 = fmaf(wsc[j], qk_rp_dot<EPL>(rg[s][0], hh, hs8, lane_tbl), acc0);
-                        acc1 = fmaf(wsc[j], qk_rp_dot<EPL>(rg[s][1], hh, hs8, lane_tbl), acc1);
+                        const float w = wsc[j];
+                        acc0 = fmaf(w, qk_rp_dot<EPL>(rg[s][0], hh, hs8, lane_tbl), acc0);
+                        acc1 = fmaf(w, qk_rp_dot<EPL>(rg[s][1], hh, hs8, lane_tbl), acc1);
                     }
-                    if (n + 2 < NS) {
-                        rload(rg[s][0], n + 2, 0);
-                        rload(rg[s][1], n + 2, 1);
+                    if (n0 + s + 2 < NS) {
+                        const int en = eid[jn];
+                        rload(rg[s][0], en, r0, pn);
+                        rload(rg[s][1], en, r0 + 1, pn);
+                        if (++jn == k) { jn = 0; pn++; }
                     }
+                    if (++j == k) { j = 0; p++; }
                 }
             }
         }
-        // shared expert
-        float as0 = 0.f, as1 = 0.f;
-        for (int p0 = 0; p0 < nsp; p0 += 4) {
-#pragma unroll
-            for (int s = 0; s < 4; s++) {
-                const int p = p0 + s;
-                if (p < nsp) {
-                    const float4 xa = reinterpret_cast<const float4 *>(hsl)[swz16(p * 64 + 2 * lane)];
-                    const float4 xb = reinterpret_cast<const float4 *>(hsl)[swz16(p * 64 + 2 * lane + 1)];
-                    as0 += bf16x8_dot(sr[s][0], xa, xb);
-                    as1 += bf16x8_dot(sr[s][1], xa, xb);
-                    if (p + 4 < nsp) {
-                        sr[s][0] = ldg_nc_v4(sptr(p + 4, 0));
-                        sr[s][1] = ldg_nc_v4(sptr(p + 4, 1));
-                    }
-                }
-            }
-        }
-        acc0 += as0;
-        acc1 += as1;
         // reduce: lanes 0..15 end with row 0, lanes 16..31 with row 1
         const bool hi = lane & 16;
         float v = (hi ? acc1 : acc0) + __shfl_xor_sync(0xffffffffu, hi ? acc0 : acc1, 16);

@@ -546,7 +546,7 @@ ds4moe_status ds4moe_decode_down(const ds4moe_experts *ex, const int32_t *ids, c
     const float *h = reinterpret_cast<const float *>(w8 + W.h);
     const float *hs = reinterpret_cast<const float *>(w8 + W.hs);
     const int smem = dd_layout(k, ex->f, ex->f_shared).total;
-    const int epl = ex->f / 32 < 64 ? ex->f / 32 : 64;  // weights of a row per lane and pass
+    const int epl = dd_epl(ex->f);  // weights of a row per lane and pass
     auto kern = epl == 64 ? decode_down_kernel<64> : epl == 32 ? decode_down_kernel<32>
               : epl == 16 ? decode_down_kernel<16> : decode_down_kernel<8>;
     if (!set_smem(kern, smem)) return DS4MOE_ECUDA;
