@@ -24,6 +24,13 @@
 //    the min term; a unit is 2 output rows over all k experts and the shared
 //    expert, accumulated as out[r] = sum_j w_j (D_j h_j)[r] + (Ds hs)[r].
 //
+// Both kernels are launched with programmatic dependent launch and may start
+// while the preceding grid still runs: inputs that grid writes (ids, routing
+// weights, h) are read only after griddepcontrol.wait, through plain pointers
+// (never const __restrict__, which would let the compiler treat them as
+// read-only for the kernel's lifetime: non-coherent loads, or loads hoisted
+// above the wait).
+//
 // The method (routed experts quantized, IQ2_XXS-style gate/up, Q2_K-style
 // down, shared expert unquantized) is the ds4 news summary's "model weights"
 // section; the kernel design is this library's own.
@@ -193,8 +200,8 @@ __device__ __forceinline__ float bf16x8_dot(const uint4 w, const float4 a, const
 // (expert slot j, rows NR i ..).  Row-matrix index rr = 2 * (row - first row) + (0 gate, 1 up).
 template <int VPP, int NR>
 __global__ void __launch_bounds__(DG_THREADS, 1)
-    decode_gateup_kernel(const ExpertsDev ex, const __nv_bfloat16 *__restrict__ x, const int32_t *__restrict__ ids,
-                         int k, float *__restrict__ h_out, float *__restrict__ hs_out) {
+    decode_gateup_kernel(const ExpertsDev ex, const __nv_bfloat16 *__restrict__ x, const int32_t *ids, int k,
+                         float *__restrict__ h_out, float *__restrict__ hs_out) {
     extern __shared__ __align__(1024) uint8_t smem[];
     __shared__ float s_red[DG_WARPS];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -241,7 +248,10 @@ __global__ void __launch_bounds__(DG_THREADS, 1)
                                       float((b[p >> 1] >> (16 * (p & 1) + 8)) & 0xFF));
         const uint4 v = *reinterpret_cast<uint4 *>(hv);
 #pragma unroll
-        for (int s = 0; s < 8; s++) *reinterpret_cast<uint4 *>(tbl + e_cb * 256 + ((tid & 1) * 8 + s) * 16) = v;
+        for (int s = 0; s < 8; s++) {  // slot order rotated so a quarter-warp's 8 stores hit 8 bank groups
+            const int slot = ((s + 2 * (e_cb & 3) + (tid & 1)) & 7) + (tid & 1) * 8;
+            *reinterpret_cast<uint4 *>(tbl + e_cb * 256 + slot * 16) = v;
+        }
     }
     float m = 0.f;
 #pragma unroll
@@ -277,6 +287,8 @@ __global__ void __launch_bounds__(DG_THREADS, 1)
     }
     __syncthreads();
 
+    // the down kernel may launch as CTAs of this grid finish (it waits for the whole grid before reading h)
+    pdl_launch_dependents();
     const uint32_t lane_tbl = DG_TABLE_ABS | uint32_t((lane & 15) * 16);
     bool waited = false;
     for (int u = u_first; u < n_all; u += nW) {
@@ -347,6 +359,9 @@ __global__ void __launch_bounds__(DG_THREADS, 1)
         if (lane % (2 * LPV) == 0)
             h_out[size_t(j) * f + r0 + lane / (2 * LPV)] = silu(v * inv_xs) * (up * inv_xs);
     }
+    // every warp waits once, so this grid completes only after the router's grid: the down kernel's wait on
+    // this grid then covers the routing results too
+    if (!waited) pdl_wait();
 }
 
 // ============================================================================ down + combine
@@ -475,9 +490,8 @@ __device__ __forceinline__ void dd_slice_load(uint32_t hq_addr, uint32_t hs_addr
 
 template <int EPL>
 __global__ void __launch_bounds__(DD_THREADS, 1)
-    decode_down_kernel(const ExpertsDev ex, const float *__restrict__ h, const float *__restrict__ hs_in,
-                       const int32_t *__restrict__ ids, const float *__restrict__ wts, int k,
-                       float *__restrict__ out) {
+    decode_down_kernel(const ExpertsDev ex, const float *h, const float *hs_in, const int32_t *ids, const float *wts,
+                       int k, float *__restrict__ out) {
     extern __shared__ __align__(1024) uint8_t smem[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int d = ex.d, f = ex.f, fs = ex.fs;

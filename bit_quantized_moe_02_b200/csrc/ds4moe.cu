@@ -453,12 +453,22 @@ ds4moe_status ds4moe_route(const void *x_bf16, int T, int d, const void *w_route
     }
     DS4_CHECK_LAUNCH();
     const unsigned tg = unsigned((T + 7) / 8);
-    if (E <= 32) route_topk_kernel<1><<<tg, 256, 0, st>>>(logits, T, E, k, late_bias, ids, weights);
-    else if (E <= 64) route_topk_kernel<2><<<tg, 256, 0, st>>>(logits, T, E, k, late_bias, ids, weights);
-    else if (E <= 128) route_topk_kernel<4><<<tg, 256, 0, st>>>(logits, T, E, k, late_bias, ids, weights);
-    else if (E <= 256) route_topk_kernel<8><<<tg, 256, 0, st>>>(logits, T, E, k, late_bias, ids, weights);
-    else if (E <= 512) route_topk_kernel<16><<<tg, 256, 0, st>>>(logits, T, E, k, late_bias, ids, weights);
-    else route_topk_kernel<32><<<tg, 256, 0, st>>>(logits, T, E, k, late_bias, ids, weights);
+    cudaError_t err;
+    const int per = E <= 32 ? 1 : E <= 64 ? 2 : E <= 128 ? 4 : E <= 256 ? 8 : E <= 512 ? 16 : 32;
+    switch (per) {
+#define TOPK_CASE(P)                                                                                             \
+    case P:                                                                                                      \
+        err = launch_pdl(route_topk_kernel<P>, dim3(tg), dim3(256), 0, st, static_cast<const float *>(logits), T, \
+                         E, k, late_bias, ids, weights);                                                         \
+        break;
+        TOPK_CASE(1) TOPK_CASE(2) TOPK_CASE(4) TOPK_CASE(8) TOPK_CASE(16) TOPK_CASE(32)
+#undef TOPK_CASE
+    default: return DS4MOE_EINVAL;
+    }
+    if (err != cudaSuccess) {
+        (void)cudaGetLastError();
+        return DS4MOE_ECUDA;
+    }
     DS4_CHECK_LAUNCH();
     return DS4MOE_OK;
 }

@@ -16,6 +16,7 @@ __global__ void __launch_bounds__(256) route_logits_small_kernel(const __nv_bflo
                                                                  const float *__restrict__ bias, int E,
                                                                  float *__restrict__ logits) {
     __shared__ float part[8][ROUTE_SMALL_T];
+    pdl_launch_dependents();  // top-k may launch now; it waits for these logits before reading them
     int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int e = blockIdx.x * 2 + (warp >> 2);
     int q = warp & 3;
@@ -74,6 +75,7 @@ __global__ void __launch_bounds__(256) route_logits_tiled_kernel(const __nv_bflo
                                                                  float *__restrict__ logits) {
     __shared__ float xs[32][68];
     __shared__ float ws[32][68];
+    pdl_launch_dependents();
     int t0 = blockIdx.x * 64, e0 = blockIdx.y * 64;
     int tid = threadIdx.x;
     int tx = tid % 16, ty = tid / 16;  // thread computes tokens ty*4.., experts tx*4..
@@ -128,10 +130,16 @@ __global__ void __launch_bounds__(256) route_logits_tiled_kernel(const __nv_bflo
 
 // ---- top-k: one warp per token, E <= 32 * PER logits spread over the lanes.
 // late_bias: added here when the logits kernel did not add it (tensor-core path), else NULL.
+// logits is written by the preceding grid and read after griddepcontrol.wait: a plain pointer, not
+// const __restrict__ (which would allow non-coherent or hoisted loads).
 template <int PER>
-__global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict__ logits, int T, int E, int k,
+__global__ void __launch_bounds__(256) route_topk_kernel(const float *logits, int T, int E, int k,
                                                          const float *__restrict__ late_bias,
                                                          int32_t *__restrict__ ids, float *__restrict__ weights) {
+    // launched with programmatic dependent launch: the expert kernels that follow may start their own
+    // prologues now, and this grid waits for the logits
+    pdl_launch_dependents();
+    pdl_wait();
     int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
     if (warp >= T) return;
     const float *lg = logits + size_t(warp) * E;
