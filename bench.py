@@ -193,6 +193,25 @@ def run_reference(args, ws, rank):
 # our arm
 
 
+GATEUP_KERNEL = "decode_gateup_kernel<8, 4>"
+GATEUP_SRC = os.path.join(ROOT, "bit_quantized_moe_02_b200", "csrc", "decode_gemv.cuh")
+
+
+def gateup_traffic():
+    """DRAM bytes (read + write) of one gate/up launch from the committed ncu summary, or None when the kernel
+    source has changed since those counters were taken (the summary records the source's SHA-256)."""
+    import hashlib
+    prof = os.path.join(ROOT, "profiles", "decode_gateup_traffic.json")
+    try:
+        rec = json.load(open(prof))
+        sha = hashlib.sha256(open(GATEUP_SRC, "rb").read()).hexdigest()
+        if rec.get("kernel") == GATEUP_KERNEL and rec.get("source_sha256") == sha:
+            return rec.get("bytes_per_launch")
+    except (OSError, ValueError):
+        pass
+    return None
+
+
 def run_ours(args, ws, rank, local):
     import torch
     from bit_quantized_moe_02_b200 import ds4moe
@@ -268,13 +287,7 @@ def run_ours(args, ws, rank, local):
     dn_ms = float(np.mean([b.elapsed_time(c) for _, b, c in ev]))
     gu_bytes = gateup_bytes(wl)
     achieved = gu_bytes / (gu_ms / 1e3) / 1e9
-    traffic = None
-    prof = os.path.join(ROOT, "profiles", "decode_gateup_traffic.json")
-    if os.path.exists(prof):
-        try:
-            traffic = json.load(open(prof)).get("bytes_per_launch")
-        except Exception:
-            traffic = None
+    traffic = gateup_traffic()
 
     # ---- end to end through the public API: pinned H2D of x, forward, D2H of the output, every step ----
     n_e2e = min(DECODE_BURST, 256)
@@ -317,7 +330,7 @@ def run_ours(args, ws, rank, local):
         "gpu_launches": 4 * DECODE_BURST * args.steps,
         "layer_bytes_per_token": layer_bytes(wl),
         "achieved_layer_GBps": layer_bytes(wl) * DECODE_BURST * args.steps / (t_ms / 1e3) / 1e9,
-        "roofline": {"bound": "hbm", "kernel": "decode_gateup_iq2x_kernel<16>", "achieved": achieved,
+        "roofline": {"bound": "hbm", "kernel": GATEUP_KERNEL, "achieved": achieved,
                      "peak": hbm, "unit": "GB/s", "frac": achieved / hbm, "traffic": traffic,
                      "peak_kind": peak_kind + " (burst copy)", "algorithmic_bytes_per_launch": gu_bytes,
                      "avg_launch_ms": gu_ms, "down_kernel_avg_ms": dn_ms,
