@@ -80,16 +80,20 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     return fn;
 }
 
-bool make_token_map(CUtensorMap *m, const __half *base, uint64_t rows, uint64_t cols) {
+// Row-major 16-bit matrix [rows x cols] (cols a multiple of 64) as a 2D TMA map with a 64 x 128 box.
+bool make_tile_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, bool bf16) {
     PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
     if (!enc || !base || rows == 0 || cols % 64 || !aligned16(base)) return false;
     const cuuint64_t dims[2] = {cols, rows};
     const cuuint64_t strides[1] = {cols * 2};
     const cuuint32_t box[2] = {uint32_t(tc::BK), uint32_t(tc::NT)};
     const cuuint32_t estr[2] = {1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<__half *>(base), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base),
+               dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+bool make_token_map(CUtensorMap *m, const __half *base, uint64_t rows, uint64_t cols) {
+    return make_tile_map(m, base, rows, cols, false);
 }
 
 bool fmt_quant(int f) { return f == DS4MOE_FMT_IQ2X || f == DS4MOE_FMT_Q2K || f == DS4MOE_FMT_Q4K; }
@@ -208,22 +212,32 @@ GroupedWs grouped_ws(const ds4moe_experts *ex, int T, int k) {
 // ---- grouped launch sequence --------------------------------------------------------------------------
 
 // row_units: rows of one A matrix (f for gate/up, d for down); col_tiles: token tiles (upper bound).
-// b_tma / b_rows: the token operand as the tcgen05 kernel reads it (row-major fp16, b_rows x ga.K).
+// b_tma / b_rows: the token operand as the tcgen05 kernel reads it (row-major 16-bit, b_rows x ga.K).
+// Dense A formats (tc::FMT_F16, tc::FMT_BF16D) also take their A matrices (ga.a0, ga.a1: row_units x ga.K) by TMA.
 template <int AFMT, bool GATEUP>
-ds4moe_status launch_grouped(const GroupedArgs &ga, int row_units, int col_tiles, const __half *b_tma,
-                             uint64_t b_rows, cudaStream_t st) {
+ds4moe_status launch_grouped(const GroupedArgs &ga, int row_units, int col_tiles, const void *b_tma, uint64_t b_rows,
+                             cudaStream_t st) {
     if (row_units <= 0 || col_tiles <= 0) return DS4MOE_OK;
-    if (use_tc_grouped()) {
-        CUtensorMap tmap;
-        if (!make_token_map(&tmap, b_tma, b_rows, uint64_t(ga.K))) return DS4MOE_ECUDA;
+    bool tc_path = true;
+    if constexpr (!tc::is_dense<AFMT>()) tc_path = use_tc_grouped();
+    if (tc_path) {
+        constexpr bool bf16 = AFMT == tc::FMT_BF16D;
+        CUtensorMap tb, ta0 = {}, ta1 = {};
+        if (!make_tile_map(&tb, b_tma, b_rows, uint64_t(ga.K), bf16)) return DS4MOE_ECUDA;
+        if (tc::is_dense<AFMT>()) {
+            if (!make_tile_map(&ta0, ga.a0, uint64_t(row_units), uint64_t(ga.K), bf16)) return DS4MOE_ECUDA;
+            if (GATEUP && !make_tile_map(&ta1, ga.a1, uint64_t(row_units), uint64_t(ga.K), bf16)) return DS4MOE_ECUDA;
+        }
         auto kern = tc::grouped_tc_kernel<AFMT, GATEUP>;
         constexpr int smem = tc::Cfg<GATEUP>::SMEM;
         if (!set_smem(kern, smem)) return DS4MOE_ECUDA;
-        kern<<<dim3(row_units / tc::M, col_tiles), tc::THREADS, smem, st>>>(ga, tmap);
+        kern<<<dim3(row_units / tc::M, col_tiles), tc::THREADS, smem, st>>>(ga, tb, ta0, ta1);
     } else {
-        auto kern = grouped_mma_kernel<AFMT, GATEUP>;
-        if (!set_smem(kern, GM_SMEM)) return DS4MOE_ECUDA;
-        kern<<<dim3(GATEUP ? row_units / 64 : row_units / GM_M, col_tiles), GM_THREADS, GM_SMEM, st>>>(ga);
+        if constexpr (!tc::is_dense<AFMT>()) {
+            auto kern = grouped_mma_kernel<AFMT, GATEUP>;
+            if (!set_smem(kern, GM_SMEM)) return DS4MOE_ECUDA;
+            kern<<<dim3(GATEUP ? row_units / 64 : row_units / GM_M, col_tiles), GM_THREADS, GM_SMEM, st>>>(ga);
+        }
     }
     DS4_CHECK_LAUNCH();
     return DS4MOE_OK;
@@ -291,16 +305,21 @@ ds4moe_status run_grouped(const ds4moe_experts *ex, const void *x, int T, const 
 
     if (ex->f_shared > 0) {
         const int ct = (T + tile_n - 1) / tile_n;
+        // Shared expert, a dense bf16 SwiGLU: on the tensor-core path A and the tokens both come by TMA as bf16
+        // (x as given, hs written as bf16); the warp-MMA path dequantizes A into fp16 against x16 / fp16 hs.
+        const bool dense = use_tc_grouped();
         GroupedArgs s1 = {};
         s1.a0 = static_cast<const uint8_t *>(ex->sh_gate); s1.a1 = static_cast<const uint8_t *>(ex->sh_up);
         s1.a_stride = 0; s1.rows = ex->f_shared; s1.K = ex->d;
-        s1.b_src = x16; s1.b_colscale = xinv; s1.n_pos = T; s1.out = hs; s1.ldo = ex->f_shared;
-        s = launch_grouped<DS4MOE_FMT_BF16, true>(s1, ex->f_shared, ct, x16, T, st);
+        s1.b_src = x16; s1.b_colscale = dense ? nullptr : xinv; s1.n_pos = T; s1.out = hs; s1.ldo = ex->f_shared;
+        s = dense ? launch_grouped<tc::FMT_BF16D, true>(s1, ex->f_shared, ct, xb, T, st)
+                  : launch_grouped<DS4MOE_FMT_BF16, true>(s1, ex->f_shared, ct, x16, T, st);
         if (s != DS4MOE_OK) return s;
         GroupedArgs s2 = {};
         s2.a0 = static_cast<const uint8_t *>(ex->sh_down); s2.a_stride = 0; s2.rows = ex->d; s2.K = ex->f_shared;
         s2.b_src = hs; s2.n_pos = T; s2.out = y_shared; s2.ldo = ex->d;
-        s = launch_grouped<DS4MOE_FMT_BF16, false>(s2, ex->d, ct, hs, T, st);
+        s = dense ? launch_grouped<tc::FMT_BF16D, false>(s2, ex->d, ct, hs, T, st)
+                  : launch_grouped<DS4MOE_FMT_BF16, false>(s2, ex->d, ct, hs, T, st);
         if (s != DS4MOE_OK) return s;
     }
     return DS4MOE_OK;
@@ -441,12 +460,8 @@ ds4moe_status ds4moe_route(const void *x_bf16, int T, int d, const void *w_route
         g.a_stride = 0; g.rows = E; g.K = d;
         g.b_src = x16; g.b_colscale = xinv; g.n_pos = T;
         g.out = logits; g.ldo = E;
-        CUtensorMap tmap;
-        if (!make_token_map(&tmap, x16, uint64_t(T), uint64_t(d))) return DS4MOE_ECUDA;
-        auto kern = tc::grouped_tc_kernel<tc::FMT_F16, false>;
-        constexpr int smem = tc::Cfg<false>::SMEM;
-        if (!set_smem(kern, smem)) return DS4MOE_ECUDA;
-        kern<<<dim3(E / tc::M, (T + tc::NT - 1) / tc::NT), tc::THREADS, smem, st>>>(g, tmap);
+        const ds4moe_status rs = launch_grouped<tc::FMT_F16, false>(g, E, (T + tc::NT - 1) / tc::NT, x16, T, st);
+        if (rs != DS4MOE_OK) return rs;
         late_bias = bias;
     } else {
         route_logits_tiled_kernel<<<dim3((T + 63) / 64, (E + 63) / 64), 256, 0, st>>>(x, T, d, wr, bias, E, logits);

@@ -31,7 +31,12 @@
 namespace ds4 {
 namespace tc {
 
-constexpr int FMT_F16 = 4;  // internal: dense fp16 rows used as they are (router weights)
+// Internal A formats.  Dense operands skip the dequantizing producers: the A tiles come by 2D TMA like the
+// token tiles, and the MMA reads both as they are (A and B of one MMA have the same type).
+constexpr int FMT_F16 = 4;    // fp16 rows (router weights) with fp16 tokens
+constexpr int FMT_BF16D = 5;  // bf16 rows (shared expert) with bf16 tokens
+template <int AFMT>
+__host__ __device__ constexpr bool is_dense() { return AFMT == FMT_F16 || AFMT == FMT_BF16D; }
 
 constexpr int M = 128;          // weight rows per accumulator
 constexpr int BK = 64;          // K per pipeline stage (one 128-byte swizzle row of fp16)
@@ -118,9 +123,9 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr) {
     return d;
 }
 
-// Instruction descriptor, kind::f16: fp16 A and B (K-major), fp32 accumulator, M = 128, N = n.
-__device__ __forceinline__ uint32_t instr_desc(int n) {
-    return (1u << 4) | (uint32_t(n >> 3) << 17) | (uint32_t(M >> 4) << 24);
+// Instruction descriptor, kind::f16: A and B K-major, both fp16 (or both bf16), fp32 accumulator, M = 128, N = n.
+__device__ __forceinline__ uint32_t instr_desc(int n, bool bf16 = false) {
+    return (1u << 4) | (bf16 ? (1u << 7) | (1u << 10) : 0u) | (uint32_t(n >> 3) << 17) | (uint32_t(M >> 4) << 24);
 }
 
 __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
@@ -335,7 +340,10 @@ __device__ __forceinline__ void sp_dequant(const SPack<AFMT, GATEUP> &pk, int h,
 // ---- the kernel -------------------------------------------------------------------------------------------
 
 template <int AFMT, bool GATEUP>
-__global__ void __launch_bounds__(THREADS, 1) grouped_tc_kernel(GroupedArgs a, const __grid_constant__ CUtensorMap tmap_b) {
+__global__ void __launch_bounds__(THREADS, 1)
+    grouped_tc_kernel(GroupedArgs a, const __grid_constant__ CUtensorMap tmap_b, const __grid_constant__ CUtensorMap tmap_a0,
+                      const __grid_constant__ CUtensorMap tmap_a1) {
+    constexpr bool DENSE = is_dense<AFMT>();
     using C = Cfg<GATEUP>;
     constexpr int S = C::STAGES;
     extern __shared__ uint8_t smem_raw[];
@@ -409,12 +417,12 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_tc_kernel(GroupedArgs a, c
     if (warp == 0) {
         // ------------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            const uint32_t idesc = instr_desc(n_eff);
+            const uint32_t idesc = instr_desc(n_eff, AFMT == FMT_BF16D);
             bool ok = true;
             for (int kc = 0; kc < nk && ok; kc++) {
                 const int s = kc % S;
                 const uint32_t par = (kc / S) & 1;
-                ok = mbar_wait(full_a(s), par, abort_flag) && mbar_wait(full_b(s), par, abort_flag);
+                ok = (DENSE || mbar_wait(full_a(s), par, abort_flag)) && mbar_wait(full_b(s), par, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t st = smem_u32(smem + s * C::STAGE);
@@ -438,8 +446,13 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_tc_kernel(GroupedArgs a, c
                 const int s = kc % S;
                 const uint32_t par = ((kc / S) & 1) ^ 1;
                 if (!mbar_wait(empty(s), par, abort_flag)) break;
-                const uint32_t bst = smem_u32(smem + s * C::STAGE + (GATEUP ? 2 : 1) * A_TILE);
-                mbar_expect_tx(full_b(s), B_TILE);  // full 128-row box, rows past the tensor are zero-filled
+                const uint32_t st = smem_u32(smem + s * C::STAGE), bst = st + (GATEUP ? 2 : 1) * A_TILE;
+                // full boxes: rows past a tensor's end are zero-filled and still counted
+                mbar_expect_tx(full_b(s), B_TILE + (DENSE ? (GATEUP ? 2 : 1) * A_TILE : 0));
+                if constexpr (DENSE) {
+                    tma_load_2d(st, &tmap_a0, kc * BK, blockIdx.x * M, full_b(s));
+                    if constexpr (GATEUP) tma_load_2d(st + A_TILE, &tmap_a1, kc * BK, blockIdx.x * M, full_b(s));
+                }
                 tma_load_2d(bst, &tmap_b, kc * BK, pos0, full_b(s));
                 issued = kc + 1;
             }
@@ -454,63 +467,65 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_tc_kernel(GroupedArgs a, c
         __syncwarp();
     } else {
         // ------------------------------------------------------------------ dequantizing producers
-        constexpr int SS = SPackCfg<AFMT, GATEUP>::SS;
-        constexpr int NOUT = GATEUP ? 8 : 4;
-        const int at = tid - W_A0 * 32;  // 0 .. 255
-        const int m = GATEUP ? at >> 7 : 0;
-        const int R = GATEUP ? at & 127 : at >> 1;
-        const int h = GATEUP ? 0 : at & 1;
-        const uint8_t *mat = (GATEUP && m ? a.a1 : a.a0) + size_t(e) * a.a_stride;
-        const int row = blockIdx.x * M + R;
-        const uint8_t *tbl_lane = tbl + (lane & 7) * 16;
-        const int nss = nk / SS;
-        // packed data of PF super-stages is in flight: super-stage ss+PF-1 is requested while ss is consumed
-        constexpr int PF = SPackCfg<AFMT, GATEUP>::NW <= 20 ? 3 : 2;
-        SPack<AFMT, GATEUP> pf[PF];
-#pragma unroll
-        for (int p = 0; p < PF - 1; p++)
-            if (p < nss) sp_load<AFMT, GATEUP>(pf[p], mat, a.pa, row, h, a.K, p);
-        bool inf = false;
-        bool run = true;
-        for (int base = 0; base < nss && run; base += PF) {
-#pragma unroll
-            for (int q = 0; q < PF; q++) {
-                const int ss = base + q;
-                if (ss >= nss || !run) break;
-                if (ss + PF - 1 < nss) sp_load<AFMT, GATEUP>(pf[(q + PF - 1) % PF], mat, a.pa, row, h, a.K, ss + PF - 1);
-                const SPack<AFMT, GATEUP> &cur = pf[q];
-#pragma unroll
-                for (int jj = 0; jj < SS; jj++) {
-                    const int kc = ss * SS + jj;
-                    const int s = kc % S;
-                    const uint32_t par = ((kc / S) & 1) ^ 1;
-                    if (!mbar_wait(empty(s), par, abort_flag)) {
-                        run = false;
-                        break;
+        if constexpr (!DENSE) {
+            constexpr int SS = SPackCfg<AFMT, GATEUP>::SS;
+            constexpr int NOUT = GATEUP ? 8 : 4;
+            const int at = tid - W_A0 * 32;  // 0 .. 255
+            const int m = GATEUP ? at >> 7 : 0;
+            const int R = GATEUP ? at & 127 : at >> 1;
+            const int h = GATEUP ? 0 : at & 1;
+            const uint8_t *mat = (GATEUP && m ? a.a1 : a.a0) + size_t(e) * a.a_stride;
+            const int row = blockIdx.x * M + R;
+            const uint8_t *tbl_lane = tbl + (lane & 7) * 16;
+            const int nss = nk / SS;
+            // packed data of PF super-stages is in flight: super-stage ss+PF-1 is requested while ss is consumed
+            constexpr int PF = SPackCfg<AFMT, GATEUP>::NW <= 20 ? 3 : 2;
+            SPack<AFMT, GATEUP> pf[PF];
+    #pragma unroll
+            for (int p = 0; p < PF - 1; p++)
+                if (p < nss) sp_load<AFMT, GATEUP>(pf[p], mat, a.pa, row, h, a.K, p);
+            bool inf = false;
+            bool run = true;
+            for (int base = 0; base < nss && run; base += PF) {
+    #pragma unroll
+                for (int q = 0; q < PF; q++) {
+                    const int ss = base + q;
+                    if (ss >= nss || !run) break;
+                    if (ss + PF - 1 < nss) sp_load<AFMT, GATEUP>(pf[(q + PF - 1) % PF], mat, a.pa, row, h, a.K, ss + PF - 1);
+                    const SPack<AFMT, GATEUP> &cur = pf[q];
+    #pragma unroll
+                    for (int jj = 0; jj < SS; jj++) {
+                        const int kc = ss * SS + jj;
+                        const int s = kc % S;
+                        const uint32_t par = ((kc / S) & 1) ^ 1;
+                        if (!mbar_wait(empty(s), par, abort_flag)) {
+                            run = false;
+                            break;
+                        }
+                        uint4 o[NOUT];
+                        if constexpr (SS == 4) {
+                            if (jj == 0) sp_dequant<AFMT, GATEUP, 0>(cur, h, ss, tbl_lane, o, inf);
+                            else if (jj == 1) sp_dequant<AFMT, GATEUP, 1>(cur, h, ss, tbl_lane, o, inf);
+                            else if (jj == 2) sp_dequant<AFMT, GATEUP, 2>(cur, h, ss, tbl_lane, o, inf);
+                            else sp_dequant<AFMT, GATEUP, 3>(cur, h, ss, tbl_lane, o, inf);
+                        } else if constexpr (SS == 2) {
+                            if (jj == 0) sp_dequant<AFMT, GATEUP, 0>(cur, h, ss, tbl_lane, o, inf);
+                            else sp_dequant<AFMT, GATEUP, 1>(cur, h, ss, tbl_lane, o, inf);
+                        } else {
+                            sp_dequant<AFMT, GATEUP, 0>(cur, h, ss, tbl_lane, o, inf);
+                        }
+                        uint8_t *ast = smem + s * C::STAGE + m * A_TILE;
+    #pragma unroll
+                        for (int c = 0; c < NOUT; c++)
+                            *reinterpret_cast<uint4 *>(ast + swz(R, (GATEUP ? 0 : h * 4) + c)) = o[c];
+                        fence_proxy_async();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(full_a(s));
                     }
-                    uint4 o[NOUT];
-                    if constexpr (SS == 4) {
-                        if (jj == 0) sp_dequant<AFMT, GATEUP, 0>(cur, h, ss, tbl_lane, o, inf);
-                        else if (jj == 1) sp_dequant<AFMT, GATEUP, 1>(cur, h, ss, tbl_lane, o, inf);
-                        else if (jj == 2) sp_dequant<AFMT, GATEUP, 2>(cur, h, ss, tbl_lane, o, inf);
-                        else sp_dequant<AFMT, GATEUP, 3>(cur, h, ss, tbl_lane, o, inf);
-                    } else if constexpr (SS == 2) {
-                        if (jj == 0) sp_dequant<AFMT, GATEUP, 0>(cur, h, ss, tbl_lane, o, inf);
-                        else sp_dequant<AFMT, GATEUP, 1>(cur, h, ss, tbl_lane, o, inf);
-                    } else {
-                        sp_dequant<AFMT, GATEUP, 0>(cur, h, ss, tbl_lane, o, inf);
-                    }
-                    uint8_t *ast = smem + s * C::STAGE + m * A_TILE;
-#pragma unroll
-                    for (int c = 0; c < NOUT; c++)
-                        *reinterpret_cast<uint4 *>(ast + swz(R, (GATEUP ? 0 : h * 4) + c)) = o[c];
-                    fence_proxy_async();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(full_a(s));
                 }
             }
+            if (inf) set_device_error(DS4MOE_EDEVICE);
         }
-        if (inf) set_device_error(DS4MOE_EDEVICE);
 
         // ------------------------------------------------------------------ epilogue (warps 4..7)
         if (warp < W_A0 + 4) {
@@ -526,7 +541,6 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_tc_kernel(GroupedArgs a, c
                     if constexpr (GATEUP) {
                         uint32_t u[32];
                         tmem_ld32(tq + NT + c0, u);
-                        __half *out = reinterpret_cast<__half *>(a.out);
                         bool overflow = false;
 #pragma unroll
                         for (int i = 0; i < 32; i++) {
@@ -535,8 +549,14 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_tc_kernel(GroupedArgs a, c
                                 const float sc = s_colsc[n];
                                 const float gv = __uint_as_float(g[i]) * sc, uv = __uint_as_float(u[i]) * sc;
                                 const float hv = silu(gv) * uv;
-                                overflow |= !(fabsf(hv) <= 65504.f);
-                                out[size_t(pos0 + n) * a.ldo + blockIdx.x * M + r] = __float2half(hv);
+                                const size_t o = size_t(pos0 + n) * a.ldo + blockIdx.x * M + r;
+                                if constexpr (AFMT == FMT_BF16D) {
+                                    overflow |= !isfinite(hv);
+                                    reinterpret_cast<__nv_bfloat16 *>(a.out)[o] = __float2bfloat16_rn(hv);
+                                } else {
+                                    overflow |= !(fabsf(hv) <= 65504.f);
+                                    reinterpret_cast<__half *>(a.out)[o] = __float2half(hv);
+                                }
                             }
                         }
                         if (overflow) set_device_error(DS4MOE_EDEVICE);
