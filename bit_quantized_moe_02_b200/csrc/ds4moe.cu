@@ -96,6 +96,21 @@ bool make_token_map(CUtensorMap *m, const __half *base, uint64_t rows, uint64_t 
     return make_tile_map(m, base, rows, cols, false);
 }
 
+// One plane of E prepared matrices as a 3D byte map: (row_bytes, rows, E), expert stride in bytes; box
+// (box_bytes, 128 rows, 1 expert), no swizzle.
+bool make_plane_map(CUtensorMap *m, const void *base, uint64_t row_bytes, uint64_t rows, uint64_t E,
+                    uint64_t expert_stride, uint32_t box_bytes) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc || !base || !aligned16(base) || row_bytes % 16 || expert_stride % 16 || box_bytes % 16) return false;
+    const cuuint64_t dims[3] = {row_bytes, rows, E};
+    const cuuint64_t strides[2] = {row_bytes, expert_stride};
+    const cuuint32_t box[3] = {box_bytes, uint32_t(tc::M), 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool fmt_quant(int f) { return f == DS4MOE_FMT_IQ2X || f == DS4MOE_FMT_Q2K || f == DS4MOE_FMT_Q4K; }
 
 ds4moe_status check_experts(const ds4moe_experts *ex) {
@@ -228,10 +243,25 @@ ds4moe_status launch_grouped(const GroupedArgs &ga, int row_units, int col_tiles
             if (!make_tile_map(&ta0, ga.a0, uint64_t(row_units), uint64_t(ga.K), bf16)) return DS4MOE_ECUDA;
             if (GATEUP && !make_tile_map(&ta1, ga.a1, uint64_t(row_units), uint64_t(ga.K), bf16)) return DS4MOE_ECUDA;
         }
+        CUtensorMap p0 = {}, p1 = {}, p2 = {}, p3 = {};
+        if constexpr (tc::PackTma<AFMT, GATEUP>::ON) {
+            const uint64_t K = uint64_t(ga.K), R = uint64_t(row_units), E = uint64_t(ga.n_mats);
+            bool ok;
+            if constexpr (AFMT == DS4MOE_FMT_IQ2X) {  // index and sign planes (K / 8 bytes per row) of gate and up
+                ok = make_plane_map(&p0, ga.a0 + ga.pa.off[0], K / 8, R, E, ga.a_stride, 32) &&
+                     make_plane_map(&p1, ga.a0 + ga.pa.off[1], K / 8, R, E, ga.a_stride, 32) &&
+                     make_plane_map(&p2, ga.a1 + ga.pa.off[0], K / 8, R, E, ga.a1_stride, 32) &&
+                     make_plane_map(&p3, ga.a1 + ga.pa.off[1], K / 8, R, E, ga.a1_stride, 32);
+            } else {  // Q2K codes (K / 4 bytes per row) and scales (K / 16)
+                ok = make_plane_map(&p0, ga.a0 + ga.pa.off[0], K / 4, R, E, ga.a_stride, 64) &&
+                     make_plane_map(&p1, ga.a0 + ga.pa.off[1], K / 16, R, E, ga.a_stride, 16);
+            }
+            if (!ok) return DS4MOE_ECUDA;
+        }
         auto kern = tc::grouped_tc_kernel<AFMT, GATEUP>;
-        constexpr int smem = tc::Cfg<GATEUP>::SMEM;
+        constexpr int smem = tc::Cfg<AFMT, GATEUP>::SMEM;
         if (!set_smem(kern, smem)) return DS4MOE_ECUDA;
-        kern<<<dim3(row_units / tc::M, col_tiles), tc::THREADS, smem, st>>>(ga, tb, ta0, ta1);
+        kern<<<dim3(row_units / tc::M, col_tiles), tc::THREADS, smem, st>>>(ga, tb, ta0, ta1, p0, p1, p2, p3);
     } else {
         if constexpr (!tc::is_dense<AFMT>()) {
             auto kern = grouped_mma_kernel<AFMT, GATEUP>;
@@ -283,7 +313,8 @@ ds4moe_status run_grouped(const ds4moe_experts *ex, const void *x, int T, const 
 
     // routed GEMM-1: gate/up -> h16
     GroupedArgs g1 = {};
-    g1.a0 = D.gate; g1.a1 = D.up; g1.a_stride = D.gate_stride; g1.pa = D.pg;
+    g1.a0 = D.gate; g1.a1 = D.up; g1.a_stride = D.gate_stride; g1.a1_stride = D.up_stride; g1.pa = D.pg;
+    g1.n_mats = ex->E;
     g1.rows = ex->f; g1.K = ex->d; g1.codebook = ex->codebook;
     g1.b_src = x16; g1.b_rowidx = perm_tok; g1.b_colscale = xinv;
     g1.tile_e = tile_e; g1.tile_pos0 = tile_pos0; g1.tile_cnt = tile_cnt; g1.n_tiles = meta;
@@ -295,7 +326,7 @@ ds4moe_status run_grouped(const ds4moe_experts *ex, const void *x, int T, const 
 
     // routed GEMM-2: down -> y_perm (scaled by the routing weight)
     GroupedArgs g2 = {};
-    g2.a0 = D.down; g2.a_stride = D.down_stride; g2.pa = D.pd; g2.rows = ex->d; g2.K = ex->f;
+    g2.a0 = D.down; g2.a_stride = D.down_stride; g2.pa = D.pd; g2.rows = ex->d; g2.K = ex->f; g2.n_mats = ex->E;
     g2.b_src = h16; g2.b_rowidx = nullptr; g2.b_colscale = nullptr;
     g2.tile_e = tile_e; g2.tile_pos0 = tile_pos0; g2.tile_cnt = tile_cnt; g2.n_tiles = meta;
     g2.pos_weight = perm_w; g2.out = y_perm; g2.ldo = ex->d;

@@ -25,7 +25,9 @@ constexpr int GM_SMEM = 2 * GM_A_BYTES + 2 * GM_B_BYTES + GM_TABLE_BYTES;
 struct GroupedArgs {
     const uint8_t *a0;  // gate (GATEUP) or down matrix of expert 0; dense bf16 matrix for the shared expert
     const uint8_t *a1;  // up matrix of expert 0 (GATEUP)
-    uint64_t a_stride;  // bytes between experts
+    uint64_t a_stride;  // bytes between experts (a0)
+    uint64_t a1_stride; // bytes between experts (a1)
+    int n_mats;         // experts (matrices) behind a0 / a1
     Planes pa;
     int rows;  // rows of one A matrix
     int K;
@@ -232,7 +234,7 @@ __global__ void __launch_bounds__(GM_THREADS) grouped_mma_kernel(GroupedArgs a) 
     int arow;
     if constexpr (GATEUP) {
         const int q = R >> 4, w = R & 15;
-        amat = (w < 8 ? a.a0 : a.a1) + size_t(e) * a.a_stride;
+        amat = w < 8 ? a.a0 + size_t(e) * a.a_stride : a.a1 + size_t(e) * a.a1_stride;
         arow = blockIdx.x * 64 + 8 * q + (w & 7);
     } else {
         amat = a.a0 + size_t(e) * a.a_stride;

@@ -49,13 +49,26 @@ constexpr int B_TILE = NT * BK * 2;  // 16 KB
 constexpr int TABLE_BYTES = 256 * 8 * 16;
 constexpr long long WAIT_NS = 2000000000LL;  // 2 s bound on any single wait
 
-template <bool GATEUP>
+// Packed A planes streamed by TMA (3D maps: plane bytes x rows x experts) into a 2-slot shared-memory ring, one
+// slot per 256-wide K block of the tile's 128 rows: IQ2X gate/up (index and sign planes of both matrices, 16 KB)
+// and Q2K down (code and scale planes, 10 KB).  The producers read them there; the few per-block scalars
+// (group scales, d, dmin) stay plain global loads.  Other formats load their packed data into registers.
+template <int AFMT, bool GATEUP>
+struct PackTma {
+    static constexpr bool ON = (AFMT == DS4MOE_FMT_IQ2X && GATEUP) || (AFMT == DS4MOE_FMT_Q2K && !GATEUP);
+    static constexpr int SLOT = AFMT == DS4MOE_FMT_IQ2X ? 4 * M * 32 : M * 64 + M * 16;
+    static constexpr int NSLOT = ON ? 2 : 0;
+};
+
+template <int AFMT, bool GATEUP>
 struct Cfg {
-    static constexpr int STAGES = 4;
+    static constexpr int STAGES = (AFMT == DS4MOE_FMT_IQ2X && GATEUP) ? 3 : 4;
     static constexpr int STAGE = (GATEUP ? 2 : 1) * A_TILE + B_TILE;
     static constexpr int TMEM_COLS = GATEUP ? 256 : 128;
-    static constexpr int TABLE_OFF = STAGES * STAGE;
+    static constexpr int PRING_OFF = STAGES * STAGE;
+    static constexpr int TABLE_OFF = PRING_OFF + PackTma<AFMT, GATEUP>::NSLOT * PackTma<AFMT, GATEUP>::SLOT;
     static constexpr int SMEM = TABLE_OFF + TABLE_BYTES + 1024;  // + alignment slack
+    static_assert(SMEM <= 232448, "shared memory");
 };
 
 // ---- PTX wrappers -----------------------------------------------------------------------------------------
@@ -158,6 +171,15 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
             dst),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
+        : "memory");
+}
+// 3D TMA tensor load (tile mode, no multicast): box at (c0 = byte, c1 = row, c2 = expert)
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, int c0, int c1, int c2,
+                                            uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+        "[%5];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
         : "memory");
 }
 __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
@@ -342,14 +364,17 @@ __device__ __forceinline__ void sp_dequant(const SPack<AFMT, GATEUP> &pk, int h,
 template <int AFMT, bool GATEUP>
 __global__ void __launch_bounds__(THREADS, 1)
     grouped_tc_kernel(GroupedArgs a, const __grid_constant__ CUtensorMap tmap_b, const __grid_constant__ CUtensorMap tmap_a0,
-                      const __grid_constant__ CUtensorMap tmap_a1) {
+                      const __grid_constant__ CUtensorMap tmap_a1, const __grid_constant__ CUtensorMap pmap0,
+                      const __grid_constant__ CUtensorMap pmap1, const __grid_constant__ CUtensorMap pmap2,
+                      const __grid_constant__ CUtensorMap pmap3) {
     constexpr bool DENSE = is_dense<AFMT>();
-    using C = Cfg<GATEUP>;
+    using PT = PackTma<AFMT, GATEUP>;
+    using C = Cfg<AFMT, GATEUP>;
     constexpr int S = C::STAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *tbl = smem + C::TABLE_OFF;
-    __shared__ __align__(8) uint64_t bars[3 * 4 + 1];  // full_a[S], full_b[S], empty[S], accum
+    __shared__ __align__(8) uint64_t bars[3 * 4 + 1 + 4];  // full_a[S], full_b[S], empty[S], accum, packed ring
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
     __shared__ float s_colsc[NT];
@@ -374,6 +399,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     auto full_b = [&](int s) { return smem_u32(&bars[4 + s]); };
     auto empty = [&](int s) { return smem_u32(&bars[8 + s]); };
     const uint32_t accum_bar = smem_u32(&bars[12]);
+    auto full_p = [&](int s) { return smem_u32(&bars[13 + s]); };
+    auto empty_p = [&](int s) { return smem_u32(&bars[15 + s]); };
+    const int nss_p = a.K / QK;  // packed-ring blocks
 
     if (tid == 0) {
         for (int s = 0; s < S; s++) {
@@ -382,6 +410,10 @@ __global__ void __launch_bounds__(THREADS, 1)
             mbar_init(empty(s), 1);
         }
         mbar_init(accum_bar, 1);
+        for (int s = 0; s < 2; s++) {
+            mbar_init(full_p(s), 1);
+            mbar_init(empty_p(s), N_WA);
+        }
         s_abort = 0;
         fence_mbar_init();
     }
@@ -464,17 +496,123 @@ __global__ void __launch_bounds__(THREADS, 1)
                     }
             }
         }
+        if constexpr (PT::ON) {
+            // ------------------------------------------------------------------ packed A planes: 3D TMA copies
+            if (warp == W_B0 + 1 && lane == 0) {
+                int issued = 0;
+                const int row0 = blockIdx.x * M;
+                for (int ss = 0; ss < nss_p; ss++) {
+                    const int sl = ss & 1;
+                    if (!mbar_wait(empty_p(sl), ((ss >> 1) & 1) ^ 1, abort_flag)) break;
+                    const uint32_t dst = smem_u32(smem + C::PRING_OFF + sl * PT::SLOT);
+                    mbar_expect_tx(full_p(sl), PT::SLOT);
+                    if constexpr (AFMT == DS4MOE_FMT_IQ2X) {  // gate idx, gate sgn, up idx, up sgn: 32 B x 128 rows
+                        tma_load_3d(dst, &pmap0, ss * 32, row0, e, full_p(sl));
+                        tma_load_3d(dst + M * 32, &pmap1, ss * 32, row0, e, full_p(sl));
+                        tma_load_3d(dst + 2 * M * 32, &pmap2, ss * 32, row0, e, full_p(sl));
+                        tma_load_3d(dst + 3 * M * 32, &pmap3, ss * 32, row0, e, full_p(sl));
+                    } else {  // Q2K codes 64 B x 128 rows, scales 16 B x 128 rows
+                        tma_load_3d(dst, &pmap0, ss * 64, row0, e, full_p(sl));
+                        tma_load_3d(dst + M * 64, &pmap1, ss * 16, row0, e, full_p(sl));
+                    }
+                    issued = ss + 1;
+                }
+                if (*abort_flag) {  // let copies in flight land before the shared memory is released (bounded)
+                    const uint64_t t0 = globaltimer();
+                    for (int ss = max(0, issued - 2); ss < issued; ss++)
+                        while (!mbar_try_wait(full_p(ss & 1), (ss >> 1) & 1) && globaltimer() - t0 < uint64_t(WAIT_NS)) {
+                        }
+                }
+            }
+        }
         __syncwarp();
     } else {
         // ------------------------------------------------------------------ dequantizing producers
-        if constexpr (!DENSE) {
+        if constexpr (PT::ON) {
+            constexpr int NOUT = GATEUP ? 8 : 4;
+            const int at = tid - W_A0 * 32;  // 0 .. 255
+            const int m = GATEUP ? at >> 7 : 0;
+            const int R = GATEUP ? at & 127 : at >> 1;
+            const int h = GATEUP ? 0 : at & 1;
+            const uint8_t *mat = GATEUP && m ? a.a1 + size_t(e) * a.a1_stride : a.a0 + size_t(e) * a.a_stride;
+            const size_t rowb = size_t(blockIdx.x * M + R) * nss_p;  // block index of the row's first block
+            const uint8_t *tbl_lane = tbl + (lane & 7) * 16;
+            // per-block scalars two blocks ahead: IQ2X group scales and d, Q2K d | dmin << 16
+            auto sload = [&](uint32_t &w0, uint32_t &w1, int ss) {
+                if (ss >= nss_p) return;
+                if constexpr (AFMT == DS4MOE_FMT_IQ2X) {
+                    w0 = ldg_nc_u32(mat + a.pa.off[2] + (rowb + ss) * 4);
+                    w1 = *reinterpret_cast<const uint16_t *>(mat + a.pa.off[3] + (rowb + ss) * 2);
+                } else {
+                    w0 = ldg_nc_u32(mat + a.pa.off[2] + (rowb + ss) * 4);
+                    w1 = 0;
+                }
+            };
+            uint32_t s00 = 0, s01 = 0, s10 = 0, s11 = 0, s20 = 0, s21 = 0;
+            sload(s00, s01, 0);
+            sload(s10, s11, 1);
+            bool inf = false, run = true;
+            for (int ss = 0; ss < nss_p && run; ss++) {
+                sload(s20, s21, ss + 2);
+                const int sl = ss & 1;
+                if (!mbar_wait(full_p(sl), (ss >> 1) & 1, abort_flag)) break;
+                const uint8_t *slot = smem + C::PRING_OFF + sl * PT::SLOT;
+                SPack<AFMT, GATEUP> cur;
+                if constexpr (AFMT == DS4MOE_FMT_IQ2X) {
+                    const uint4 *ip = reinterpret_cast<const uint4 *>(slot + m * 2 * M * 32 + R * 32);
+                    const uint4 *sp = reinterpret_cast<const uint4 *>(slot + m * 2 * M * 32 + M * 32 + R * 32);
+                    const uint4 i0 = ip[0], i1 = ip[1], g0 = sp[0], g1 = sp[1];
+                    cur.w[0] = i0.x; cur.w[1] = i0.y; cur.w[2] = i0.z; cur.w[3] = i0.w;
+                    cur.w[4] = i1.x; cur.w[5] = i1.y; cur.w[6] = i1.z; cur.w[7] = i1.w;
+                    cur.w[8] = g0.x; cur.w[9] = g0.y; cur.w[10] = g0.z; cur.w[11] = g0.w;
+                    cur.w[12] = g1.x; cur.w[13] = g1.y; cur.w[14] = g1.z; cur.w[15] = g1.w;
+                    cur.w[16] = s00; cur.w[17] = s01;
+                } else {
+                    const uint8_t *q = slot + R * 64 + h * 8;
+#pragma unroll
+                    for (int j = 0; j < 4; j++) {
+                        const uint2 v = *reinterpret_cast<const uint2 *>(q + 16 * j);
+                        cur.w[2 * j] = v.x; cur.w[2 * j + 1] = v.y;
+                    }
+                    const uint4 sc = *reinterpret_cast<const uint4 *>(slot + M * 64 + R * 16);
+                    cur.w[8] = sc.x; cur.w[9] = sc.y; cur.w[10] = sc.z; cur.w[11] = sc.w;
+                    cur.w[12] = s00;
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(empty_p(sl));  // the slot may be refilled
+                s00 = s10; s01 = s11; s10 = s20; s11 = s21;
+#pragma unroll
+                for (int jj = 0; jj < 4; jj++) {
+                    const int kc = ss * 4 + jj;
+                    const int s = kc % S;
+                    const uint32_t par = ((kc / S) & 1) ^ 1;
+                    if (!mbar_wait(empty(s), par, abort_flag)) {
+                        run = false;
+                        break;
+                    }
+                    uint4 o[NOUT];
+                    if (jj == 0) sp_dequant<AFMT, GATEUP, 0>(cur, h, ss, tbl_lane, o, inf);
+                    else if (jj == 1) sp_dequant<AFMT, GATEUP, 1>(cur, h, ss, tbl_lane, o, inf);
+                    else if (jj == 2) sp_dequant<AFMT, GATEUP, 2>(cur, h, ss, tbl_lane, o, inf);
+                    else sp_dequant<AFMT, GATEUP, 3>(cur, h, ss, tbl_lane, o, inf);
+                    uint8_t *ast = smem + s * C::STAGE + m * A_TILE;
+#pragma unroll
+                    for (int c = 0; c < NOUT; c++)
+                        *reinterpret_cast<uint4 *>(ast + swz(R, (GATEUP ? 0 : h * 4) + c)) = o[c];
+                    fence_proxy_async();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(full_a(s));
+                }
+            }
+            if (inf) set_device_error(DS4MOE_EDEVICE);
+        } else if constexpr (!DENSE) {
             constexpr int SS = SPackCfg<AFMT, GATEUP>::SS;
             constexpr int NOUT = GATEUP ? 8 : 4;
             const int at = tid - W_A0 * 32;  // 0 .. 255
             const int m = GATEUP ? at >> 7 : 0;
             const int R = GATEUP ? at & 127 : at >> 1;
             const int h = GATEUP ? 0 : at & 1;
-            const uint8_t *mat = (GATEUP && m ? a.a1 : a.a0) + size_t(e) * a.a_stride;
+            const uint8_t *mat = GATEUP && m ? a.a1 + size_t(e) * a.a1_stride : a.a0 + size_t(e) * a.a_stride;
             const int row = blockIdx.x * M + R;
             const uint8_t *tbl_lane = tbl + (lane & 7) * 16;
             const int nss = nk / SS;
