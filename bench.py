@@ -295,18 +295,20 @@ def run_ours(args, ws, rank, local):
     out_host = torch.empty((1, s.d), dtype=torch.float32).pin_memory()
     x_dev = torch.empty((1, s.d), dtype=torch.int16, device="cuda")
     with torch.cuda.stream(stream):
-        for i in range(8):
+        for i in range(16):
             layers[i % LAYERS].forward(x_dev.view(torch.bfloat16))
         stream.synchronize()
-        barrier(ws)
-        t0 = time.perf_counter()
-        for i in range(n_e2e):
-            x_dev.copy_(x_host[i:i + 1], non_blocking=True)
-            o = layers[i % LAYERS].forward(x_dev.view(torch.bfloat16))
-            out_host.copy_(o, non_blocking=True)
-            stream.synchronize()
-        e2e_s = time.perf_counter() - t0
-    e2e_s = max_over_ranks(e2e_s, ws)
+        runs = []
+        for _ in range(3):  # host wall clock on a shared machine: the median of three 256-token runs
+            barrier(ws)
+            t0 = time.perf_counter()
+            for i in range(n_e2e):
+                x_dev.copy_(x_host[i:i + 1], non_blocking=True)
+                o = layers[i % LAYERS].forward(x_dev.view(torch.bfloat16))
+                out_host.copy_(o, non_blocking=True)
+                stream.synchronize()
+            runs.append(max_over_ranks(time.perf_counter() - t0, ws))
+        e2e_s = sorted(runs)[1]
     e2e_value = n_e2e * ws / e2e_s
 
     # ---- prefill: T=4096 grouped path (one layer, eager) ----
@@ -338,7 +340,8 @@ def run_ours(args, ws, rank, local):
                      "down_kernel_GBps": (layer_bytes(wl) - gu_bytes - s.router_bytes) / (dn_ms / 1e3) / 1e9},
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": s.d * 2, "d2h_bytes_per_step": s.d * 4,
-                "note": "one token per step through DeviceLayer.forward (route + decode), eager, sync per token"},
+                "note": "one token per step through DeviceLayer.forward (route + decode), eager, sync per token; "
+                        "median of 3 runs of 256 tokens"},
         "clocks": clk.summary(),
         "prefill": prefill,
         "setup_s": setup_s,

@@ -5,6 +5,8 @@
 #include <stdio.h>
 #include <stdlib.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "decode_gemv.cuh"
 #include "grouped_mma.cuh"
@@ -38,10 +40,32 @@ int num_sms() {
     return n;
 }
 
-// Opt in to the dynamic shared memory a kernel needs (static + dynamic above 48 KB needs the attribute).
+// Opt in to the dynamic shared memory a kernel needs (static + dynamic above 48 KB needs the attribute).  The
+// attribute is per function and device and stays set, so each (kernel, device) pair is configured once for the
+// largest size asked so far: a per-launch cudaFuncSetAttribute is a measurable share of a decode call.
 template <typename Kern>
 bool set_smem(Kern k, int bytes) {
-    return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
+    struct Entry {
+        const void *fn;
+        int dev, bytes;
+    };
+    static Entry cache[256];
+    static int n = 0;
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    const void *fn = reinterpret_cast<const void *>(k);
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < n; i++)
+        if (cache[i].fn == fn && cache[i].dev == dev) {
+            if (cache[i].bytes >= bytes) return true;
+            if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
+            cache[i].bytes = bytes;
+            return true;
+        }
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
+    if (n < 256) cache[n++] = Entry{fn, dev, bytes};
+    return true;
 }
 
 // Launch with programmatic dependent launch enabled (the kernel calls pdl_wait before consuming

@@ -115,9 +115,8 @@ def route(x: torch.Tensor, wr: torch.Tensor, bias: Optional[torch.Tensor], k: in
           ids: Optional[torch.Tensor] = None, weights: Optional[torch.Tensor] = None):
     T, d = x.shape
     E = wr.shape[0]
-    need = int(lib().ds4moe_route_workspace_size(T, d, E))
-    if ws is None or ws.numel() < need:
-        ws = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
+    if ws is None:  # a caller-provided workspace is checked against the required size by the library
+        ws = torch.empty(max(int(lib().ds4moe_route_workspace_size(T, d, E)), 1), dtype=torch.uint8, device=x.device)
     ids = torch.empty((T, k), dtype=torch.int32, device=x.device) if ids is None else ids
     weights = torch.empty((T, k), dtype=torch.float32, device=x.device) if weights is None else weights
     _check(lib().ds4moe_route(_p(x), T, d, _p(wr), _p(bias), E, k, _p(ids), _p(weights), _p(ws), ws.numel(),
@@ -234,15 +233,22 @@ class DeviceLayer:
         self.ws = torch.empty(need, dtype=torch.uint8, device=self.device)
         self.route_ws = torch.empty(max(int(lib().ds4moe_route_workspace_size(T, s.d, s.E)), 1), dtype=torch.uint8,
                                     device=self.device)
+        self.ids_buf = torch.empty((T, s.k), dtype=torch.int32, device=self.device)
+        self.w_buf = torch.empty((T, s.k), dtype=torch.float32, device=self.device)
         self.max_tokens = T
 
-    def route(self, x: torch.Tensor):
-        return route(x, self.wr, self.bias, self.shape.k, ws=self.route_ws)
+    def route(self, x: torch.Tensor, ids: Optional[torch.Tensor] = None, weights: Optional[torch.Tensor] = None):
+        return route(x, self.wr, self.bias, self.shape.k, ws=self.route_ws, ids=ids, weights=weights)
 
     def forward(self, x: torch.Tensor, out: Optional[torch.Tensor] = None, return_routing: bool = False):
+        """Layer output for x [T, d] (bf16): route, experts, combine.  Without return_routing the routing goes
+        to buffers owned by the layer (reused by the next call on the same stream order)."""
         T = x.shape[0]
         self.reserve(T)
-        ids, w = self.route(x)
+        if return_routing:
+            ids, w = self.route(x)
+        else:
+            ids, w = self.route(x, ids=self.ids_buf[:T], weights=self.w_buf[:T])
         out = expert_ffn_decode(self.ex, x, ids, w, self.ws, out=out)
         return (out, ids, w) if return_routing else out
 
