@@ -77,3 +77,29 @@ def test_host_side_argument_checks():
     assert lib.ds4moe_expert_ffn_grouped(ctypes.byref(bad), fake, 4, fake, fake, 2, fake, fake, None, fake, 1 << 30,
                                          None) == 1
     assert lib.ds4moe_last_device_error(None, None) == 1
+
+
+def test_decode_gemv_limits_checked_on_host():
+    """The single-token GEMV halves refuse layers outside their limits before any launch: d must be 256 times a
+    power of two up to 8192, f likewise, gate/up IQ2X with Q2K down, k <= 32; the combined decode call then
+    runs the grouped path instead (its own checks)."""
+    lib = ds4moe.lib()
+    fake = ctypes.c_void_p(1 << 20)
+
+    def experts(d, f, fmt_gate=0, fmt_down=1, fs=0):
+        return ds4moe.Experts(d, f, 8, fs, fmt_gate, fmt_gate, fmt_down, 1 << 20, 1 << 22, 1 << 24, 1 << 26,
+                              1 << 26, 1 << 26, 1 << 23, None, None, None)
+
+    for d, f in ((768, 512), (256, 768), (16384, 512)):  # not 256 * 2^i, or d beyond 8192
+        ex = experts(d, f)
+        assert lib.ds4moe_decode_gateup(ctypes.byref(ex), fake, fake, 2, fake, 1 << 30, None) == 2, (d, f)
+        assert lib.ds4moe_decode_down(ctypes.byref(ex), fake, fake, 2, fake, fake, 1 << 30, None) == 2, (d, f)
+    q4 = experts(512, 512, fmt_gate=2, fmt_down=2)  # Q4K has no GEMV kernel
+    assert lib.ds4moe_decode_gateup(ctypes.byref(q4), fake, fake, 2, fake, 1 << 30, None) == 2
+    ex = experts(512, 512)
+    assert lib.ds4moe_decode_gateup(ctypes.byref(ex), fake, fake, 40, fake, 1 << 30, None) == 1  # k > E
+    # workspace: h (k*f floats) and the shared expert's h, each rounded to 256 bytes
+    need = (2 * 512 * 4 + 255) // 256 * 256 + 256
+    assert lib.ds4moe_decode_gateup(ctypes.byref(ex), fake, fake, 2, fake, need - 1, None) == 4
+    assert lib.ds4moe_expert_ffn_decode_noalloc(ctypes.byref(experts(768, 512)), fake, fake, fake, 2, fake,
+                                                None) == 2
