@@ -10,18 +10,23 @@
 //               producers and finally signals the epilogue.
 //   warp 1      loads the tile's token rows (permuted fp16 activations or
 //               SwiGLU outputs, contiguous per expert) with one 2D TMA tensor
-//               copy per stage into a 128B-swizzled K-major stage.
-//   warps 4-11  stream the packed 2-bit (or 4-bit) blocks, dequantize them in
-//               registers (shared-memory codebook / sign-bit XOR / fp16 scale)
-//               and write fp16 tiles in the same swizzled K-major layout the
-//               MMA descriptor describes.  Warps 4-7 then run the epilogue:
-//               tcgen05.ld the accumulators, SwiGLU (gate/up) or routing-weight
-//               scaling (down), coalesced stores.
+//               copy per stage into a 128B-swizzled K-major stage; for dense
+//               formats (router fp16, shared-expert bf16) it loads the A tiles
+//               the same way.
+//   warp 2      streams the packed IQ2X / Q2K planes of the tile's rows, one
+//               256-wide K block at a time, with 3D TMA copies into a 2-slot
+//               shared-memory ring (Q4K and bf16 producers load into registers).
+//   warps 4-11  dequantize the packed blocks in registers (shared-memory
+//               codebook / sign-bit XOR / fp16 scale) and write fp16 tiles in
+//               the same swizzled K-major layout the MMA descriptor describes.
+//               Warps 4-7 then run the epilogue: tcgen05.ld the accumulators,
+//               SwiGLU (gate/up) or routing-weight scaling (down), stores.
 //
 // Gate and up share one work item: two accumulators (TMEM columns [0,128) and
 // [128,256)) hold matching rows, so each epilogue thread owns a gate/up pair.
 // Every wait on an mbarrier is bounded; a timeout records DS4MOE_ETIMEOUT,
-// stops the CTA's roles and still frees TMEM before returning.
+// stops the CTA's roles, lets its TMA copies in flight land and still frees
+// TMEM before returning.
 #pragma once
 #include <cuda.h>
 
@@ -187,14 +192,6 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
                      bar),
                  "r"(bytes)
                  : "memory");
-}
-
-__device__ __forceinline__ void cp_async_wait_le(int n) {
-    // n is small and uniform; branch to the immediate forms
-    if (n <= 0) asm volatile("cp.async.wait_group 0;" ::: "memory");
-    else if (n == 1) asm volatile("cp.async.wait_group 1;" ::: "memory");
-    else if (n == 2) asm volatile("cp.async.wait_group 2;" ::: "memory");
-    else asm volatile("cp.async.wait_group 3;" ::: "memory");
 }
 
 // ---- A producers: packed data for a "super-stage" of SS pipeline stages is loaded one super-stage ahead ------

@@ -143,8 +143,14 @@ ds4moe_status ds4moe_dequant(ds4moe_fmt fmt, const void *prepared, const uint8_t
  * or NULL (added to the logit before the sigmoid).  Writes ids int32 [T x k]
  * (descending score, ties to the smaller id) and weights fp32 [T x k]
  * (renormalised to sum 1).  Products fp16 x bf16 are exact in fp32 and the
- * dot products accumulate in fp32.  1 <= k <= min(E, 32), E <= 1024,
- * d multiple of 256. */
+ * dot products accumulate in fp32: on CUDA cores for T <= 8 (and for E not a
+ * multiple of 128), otherwise on the tensor cores with x scaled per token by
+ * a power of two into fp16 (exact products, fp32 accumulation).  The top-k
+ * kernel is launched with programmatic dependent launch after the logits.
+ * 1 <= k <= min(E, 32), E <= 1024, d multiple of 256.  The workspace
+ * (ds4moe_route_workspace_size bytes, 256-byte aligned) holds the logits and,
+ * on the tensor-core path, the scaled activations; a smaller one is refused
+ * with DS4MOE_ENOWORKSPACE. */
 size_t ds4moe_route_workspace_size(int T, int d, int E);
 ds4moe_status ds4moe_route(const void *x_bf16, int T, int d, const void *w_router_f16, const float *bias, int E,
                            int k, int32_t *ids, float *weights, void *ws, size_t ws_bytes, ds4moe_stream stream);
