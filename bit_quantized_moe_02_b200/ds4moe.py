@@ -252,6 +252,10 @@ class DeviceLayer:
         out = expert_ffn_decode(self.ex, x, ids, w, self.ws, out=out)
         return (out, ids, w) if return_routing else out
 
+    def decode_graph(self) -> "DecodeGraph":
+        """A CUDA-graph replay of this layer's single-token decode (route + experts); see DecodeGraph."""
+        return DecodeGraph(self)
+
     def forward_grouped(self, x: torch.Tensor):
         """Prefill entry: grouped experts then combine (returns out, ids, weights, y_perm, inv_perm)."""
         s = self.shape
@@ -264,3 +268,45 @@ class DeviceLayer:
         expert_ffn_grouped(self.ex, x, ids, w, self.ws, y_perm, inv, ys)
         out = combine(y_perm, inv, ys, T, s.d, s.k)
         return out, ids, w, y_perm, inv
+
+
+class DecodeGraph:
+    """Single-token decode of one layer replayed from a CUDA graph: the router, top-k, gate/up and down launches
+    of ``DeviceLayer.forward`` for one token, captured once, so a decode step costs one graph launch on the host.
+
+    ``x`` (bf16 [1, d]) and ``out`` (fp32 [1, d]) are buffers owned by this object: write the token into ``x``
+    (or pass it to ``__call__``), replay, read ``out``.  Replays run on the current stream; consecutive replays
+    reuse the same buffers, so read ``out`` before the next one.
+    """
+
+    def __init__(self, layer: DeviceLayer):
+        s = layer.shape
+        layer.reserve(1)
+        dev = layer.device
+        self.layer = layer
+        self.x = torch.zeros((1, s.d), dtype=torch.bfloat16, device=dev)
+        self.out = torch.empty((1, s.d), dtype=torch.float32, device=dev)
+        self.ids = torch.empty((1, s.k), dtype=torch.int32, device=dev)
+        self.weights = torch.empty((1, s.k), dtype=torch.float32, device=dev)
+        side = torch.cuda.Stream(device=dev)
+        side.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(side):
+            self._record()  # eager run first: the library configures its kernels outside the capture
+            side.synchronize()
+            self.graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(self.graph, stream=side):
+                self._record()
+        torch.cuda.current_stream(dev).wait_stream(side)
+
+    def _record(self):
+        L = self.layer
+        route(self.x, L.wr, L.bias, L.shape.k, ws=L.route_ws, ids=self.ids, weights=self.weights)
+        expert_ffn_decode(L.ex, self.x, self.ids, self.weights, L.ws, out=self.out)
+
+    def __call__(self, x: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """Copy x (bf16 or int16 bits, [1, d], device or pinned host) into the input buffer if given, replay,
+        and return the output buffer."""
+        if x is not None:
+            self.x.view(torch.int16).copy_(x.view(torch.int16), non_blocking=True)
+        self.graph.replay()
+        return self.out

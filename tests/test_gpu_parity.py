@@ -183,3 +183,18 @@ def test_bad_expert_id_sets_device_error(ds4):
     ds4.expert_ffn_decode(D.ex, x, ids, w, D.ws)
     assert ds4.last_device_error() == 6
     assert ds4.last_device_error() == 0  # read clears
+
+
+def test_decode_graph_matches_eager(ds4):
+    """The graph-replayed single-token decode runs the same launches as DeviceLayer.forward: bit-identical."""
+    wl = synth.WORKLOADS["tiny"]
+    L = synth.make_layer(wl)
+    D = ds4.DeviceLayer(L, max_tokens=1)
+    x = dev(synth.activations(wl, 4, stream=11))
+    G = D.decode_graph()
+    for t in range(4):
+        want = D.forward(x[t:t + 1].view(torch.bfloat16)).clone()
+        got = G(x[t:t + 1]).clone()
+        torch.cuda.synchronize()
+        assert ds4.last_device_error() == 0
+        assert torch.equal(got, want), t
