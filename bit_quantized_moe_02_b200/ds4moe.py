@@ -281,13 +281,16 @@ class DecodeGraph:
 
     def __init__(self, layer: DeviceLayer):
         s = layer.shape
-        layer.reserve(1)
         dev = layer.device
         self.layer = layer
         self.x = torch.zeros((1, s.d), dtype=torch.bfloat16, device=dev)
         self.out = torch.empty((1, s.d), dtype=torch.float32, device=dev)
         self.ids = torch.empty((1, s.k), dtype=torch.int32, device=dev)
         self.weights = torch.empty((1, s.k), dtype=torch.float32, device=dev)
+        # workspaces of its own: the graph keeps their addresses, which a later layer.reserve() must not free
+        self.ws = torch.empty(max(workspace_size(layer.ex, 1, s.k), 1), dtype=torch.uint8, device=dev)
+        self.route_ws = torch.empty(max(int(lib().ds4moe_route_workspace_size(1, s.d, s.E)), 1), dtype=torch.uint8,
+                                    device=dev)
         side = torch.cuda.Stream(device=dev)
         side.wait_stream(torch.cuda.current_stream(dev))
         with torch.cuda.stream(side):
@@ -300,8 +303,8 @@ class DecodeGraph:
 
     def _record(self):
         L = self.layer
-        route(self.x, L.wr, L.bias, L.shape.k, ws=L.route_ws, ids=self.ids, weights=self.weights)
-        expert_ffn_decode(L.ex, self.x, self.ids, self.weights, L.ws, out=self.out)
+        route(self.x, L.wr, L.bias, L.shape.k, ws=self.route_ws, ids=self.ids, weights=self.weights)
+        expert_ffn_decode(L.ex, self.x, self.ids, self.weights, self.ws, out=self.out)
 
     def __call__(self, x: Optional[torch.Tensor] = None) -> torch.Tensor:
         """Copy x (bf16 or int16 bits, [1, d], device or pinned host) into the input buffer if given, replay,
