@@ -116,10 +116,6 @@ bool make_tile_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t col
                dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
-bool make_token_map(CUtensorMap *m, const __half *base, uint64_t rows, uint64_t cols) {
-    return make_tile_map(m, base, rows, cols, false);
-}
-
 // One plane of E prepared matrices as a 3D byte map: (row_bytes, rows, E), expert stride in bytes; box
 // (box_bytes, 128 rows, 1 expert), no swizzle.
 bool make_plane_map(CUtensorMap *m, const void *base, uint64_t row_bytes, uint64_t rows, uint64_t E,
