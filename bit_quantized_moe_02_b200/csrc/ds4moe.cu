@@ -376,6 +376,20 @@ ds4moe_status run_grouped(const ds4moe_experts *ex, const void *x, int T, const 
     return DS4MOE_OK;
 }
 
+// ---- failure-path self-test: one thread waits, through the tensor-core kernel's bounded wait, on an mbarrier
+// that nothing arrives at; the wait gives up after tc::WAIT_NS and records DS4MOE_ETIMEOUT.
+__global__ void selftest_wait_timeout_kernel() {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        tc::mbar_init(smem_u32(&bar), 1);
+        abort_flag = 0;
+        tc::fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) (void)tc::mbar_wait(smem_u32(&bar), 0, &abort_flag);
+}
+
 // ---- scratch for the allocation-free decode entry point ------------------------------------------------
 //
 // Some callers cannot hand the library a workspace: code that must not call cudaMalloc at all
@@ -679,6 +693,13 @@ ds4moe_status ds4moe_combine(const float *y_perm, const int32_t *inv_perm, const
     const uint64_t total = uint64_t(T) * (d / 4);
     const unsigned grid = unsigned(std::min<uint64_t>((total + 255) / 256, uint64_t(num_sms()) * 16));
     combine_kernel<<<grid, 256, 0, cs(stream)>>>(y_perm, inv_perm, y_shared, T, d, k, out);
+    DS4_CHECK_LAUNCH();
+    return DS4MOE_OK;
+}
+
+ds4moe_status ds4moe_selftest_wait_timeout(ds4moe_stream stream) {
+    (void)cudaGetLastError();  // report only errors raised by this call's launch
+    selftest_wait_timeout_kernel<<<1, 32, 0, cs(stream)>>>();
     DS4_CHECK_LAUNCH();
     return DS4MOE_OK;
 }

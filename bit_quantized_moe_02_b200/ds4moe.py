@@ -25,7 +25,7 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported", 3: "CUDA error", 4: 
 EXPORTS = ["ds4moe_status_string", "ds4moe_prepared_bytes", "ds4moe_prepare", "ds4moe_dequant",
            "ds4moe_route_workspace_size", "ds4moe_route", "ds4moe_workspace_size", "ds4moe_expert_ffn_decode",
            "ds4moe_expert_ffn_grouped", "ds4moe_combine", "ds4moe_last_device_error", "ds4moe_decode_gateup",
-           "ds4moe_decode_down", "ds4moe_expert_ffn_decode_noalloc"]
+           "ds4moe_decode_down", "ds4moe_expert_ffn_decode_noalloc", "ds4moe_selftest_wait_timeout"]
 
 
 class Ds4moeError(RuntimeError):
@@ -73,6 +73,7 @@ def lib():
         l.ds4moe_decode_gateup.argtypes = [ctypes.POINTER(Experts), vp, vp, i32, vp, sz, vp]
         l.ds4moe_decode_down.argtypes = [ctypes.POINTER(Experts), vp, vp, i32, vp, vp, sz, vp]
         l.ds4moe_expert_ffn_decode_noalloc.argtypes = [ctypes.POINTER(Experts), vp, vp, vp, i32, vp, vp]
+        l.ds4moe_selftest_wait_timeout.argtypes = [vp]
         _lib = l
     return _lib
 

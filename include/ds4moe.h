@@ -228,6 +228,14 @@ ds4moe_status ds4moe_expert_ffn_grouped(const ds4moe_experts *ex, const void *x_
 ds4moe_status ds4moe_combine(const float *y_perm, const int32_t *inv_perm, const float *y_shared, int T, int d,
                              int k, float *out, ds4moe_stream stream);
 
+/* Self-test of the device failure path (no counterpart in the pages): one
+ * CTA whose thread waits, through the same bounded mbarrier wait the
+ * tensor-core kernels use, on a barrier nothing arrives at.  The wait gives
+ * up after 2 s and records DS4MOE_ETIMEOUT in the device error word (read it
+ * with ds4moe_last_device_error); the context stays usable.  Asynchronous on
+ * the stream; nothing traps or faults. */
+ds4moe_status ds4moe_selftest_wait_timeout(ds4moe_stream stream);
+
 /* Synchronizes `stream`, then reads and clears the calling device's error
  * word: *code = 0 (none), or the ds4moe_status of the first device-side
  * error since the last read (DS4MOE_EDEVICE / DS4MOE_ETIMEOUT). */
