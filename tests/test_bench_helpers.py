@@ -1,0 +1,31 @@
+"""Host-side pieces of bench.py that decide what the JSON line reports (no GPU)."""
+import hashlib
+import json
+import os
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+
+
+def test_traffic_only_while_the_profiled_source_is_unchanged(tmp_path, monkeypatch):
+    rec = json.load(open(os.path.join(ROOT, "profiles", "decode_gateup_traffic.json")))
+    sha = hashlib.sha256(open(bench.GATEUP_SRC, "rb").read()).hexdigest()
+    same = rec.get("source_sha256") == sha and rec.get("kernel") == bench.GATEUP_KERNEL
+    want = rec["bytes_per_launch"] if same else None
+    assert bench.gateup_traffic() == want
+    changed = tmp_path / "decode_gemv.cuh"
+    changed.write_bytes(open(bench.GATEUP_SRC, "rb").read() + b"// changed")
+    monkeypatch.setattr(bench, "GATEUP_SRC", str(changed))
+    assert bench.gateup_traffic() is None  # counters taken on another version of the kernel: no traffic
+
+
+def test_algorithmic_bytes_of_the_decode_workload():
+    from bit_quantized_moe_02_b200 import synth
+    wl = synth.WORKLOADS["decode"]
+    s = wl.shape
+    # routed IQ2X gate + up (66 B / 256 weights) + shared bf16 gate + up + x (bf16)
+    want = s.k * 2 * s.f * s.d // 256 * 66 + 2 * s.f_shared * s.d * 2 + s.d * 2
+    assert bench.gateup_bytes(wl) == want == 68165632
