@@ -128,14 +128,18 @@ size_t ds4moe_prepared_bytes(ds4moe_fmt fmt, int rows, int cols);
  * matrix m at canonical + m*rows*(cols/256)*block_bytes) into the prepared
  * layout at prepared + m*prepared_stride.  prepared_stride >=
  * ds4moe_prepared_bytes() and a multiple of 256; prepared 256-byte aligned.
- * The block layouts are defined above; the repacking is lossless. */
+ * The block layouts are defined above; the repacking is lossless.
+ * Passage: the IQ2_XXS / Q2_K / Q4_K-style expert formats (ds4 news summary,
+ * "model weights"; upppp.jp, "asymmetric 2-bit quantization"); the prepared
+ * plane split is this library's own layout, with no counterpart there. */
 ds4moe_status ds4moe_prepare(ds4moe_fmt fmt, const void *canonical, void *prepared, int rows, int cols, int n_mats,
                              uint64_t prepared_stride, ds4moe_stream stream);
 
 /* Exact fp32 dequantization of one prepared matrix into out[rows x cols]
  * (row-major).  Every value equals the block definition evaluated in fp32:
  * all products are exact and the Q2K/Q4K subtraction rounds once, so the
- * result is bit-exact whatever the evaluation order.  Test / export call. */
+ * result is bit-exact whatever the evaluation order.  Test / export call.
+ * Passage: the same expert formats as ds4moe_prepare. */
 ds4moe_status ds4moe_dequant(ds4moe_fmt fmt, const void *prepared, const uint8_t *codebook, int rows, int cols,
                              float *out, ds4moe_stream stream);
 
@@ -150,7 +154,10 @@ ds4moe_status ds4moe_dequant(ds4moe_fmt fmt, const void *prepared, const uint8_t
  * 1 <= k <= min(E, 32), E <= 1024, d multiple of 256.  The workspace
  * (ds4moe_route_workspace_size bytes, 256-byte aligned) holds the logits and,
  * on the tensor-core path, the scaled activations; a smaller one is refused
- * with DS4MOE_ENOWORKSPACE. */
+ * with DS4MOE_ENOWORKSPACE.  Passage: the router is one of the parts left
+ * unquantized (ds4 news summary, "model weights"); the pages do not give its
+ * function, and this library reads it as the sigmoid -> top-k -> renormalise
+ * rule written at the top of this file. */
 size_t ds4moe_route_workspace_size(int T, int d, int E);
 ds4moe_status ds4moe_route(const void *x_bf16, int T, int d, const void *w_router_f16, const float *bias, int E,
                            int k, int32_t *ids, float *weights, void *ws, size_t ws_bytes, ds4moe_stream stream);
@@ -168,7 +175,11 @@ size_t ds4moe_workspace_size(const ds4moe_experts *ex, int T, int k);
  * internally (each touched expert read once).  On the GEMV path x_bf16 is read
  * before the wait on the preceding kernel (see ds4moe_decode_gateup), so x
  * must not be written by the kernel launched just before this call on the
- * same stream; ds4moe_route between the two satisfies this. */
+ * same stream; ds4moe_route between the two satisfies this.  Passage: the
+ * expert FFN with quantized routed experts and an unquantized shared expert
+ * (ds4 news summary, "model weights"; upppp.jp, "asymmetric 2-bit
+ * quantization"); single-token generation speed is the pages' headline
+ * figure (ds4 news summary, "speed benchmarks"). */
 ds4moe_status ds4moe_expert_ffn_decode(const ds4moe_experts *ex, const void *x_bf16, int B, const int32_t *ids,
                                        const float *weights, int k, float *out, void *ws, size_t ws_bytes,
                                        ds4moe_stream stream);
@@ -193,7 +204,7 @@ ds4moe_status ds4moe_decode_down(const ds4moe_experts *ex, const int32_t *ids, c
 /* Single-token decode without a caller workspace, for callers that cannot
  * allocate device memory at all: an engine whose memory planner has taken all
  * of HBM and forbids further allocation, or a plugin host that exposes no
- * allocator.  The paper has no counterpart: this is a library convenience.
+ * allocator.  The pages have no counterpart: this is a library convenience.
  * Same computation and arguments as ds4moe_expert_ffn_decode with B = 1 (and
  * the same layer limits as ds4moe_decode_gateup), but the scratch comes from
  * a 1 MiB array compiled into the library, which every GPU that loads the
@@ -218,13 +229,18 @@ ds4moe_status ds4moe_expert_ffn_decode_noalloc(const ds4moe_experts *ex, const v
  *   inv_perm int32 [T*k]:   inv_perm[t*k + j] = p,
  *   y_shared fp32 [T x d]:  the shared expert's output (may be NULL iff the
  *           layer has no shared expert).
- * Follow with ds4moe_combine. */
+ * Follow with ds4moe_combine.  Passage: the same expert FFN as
+ * ds4moe_expert_ffn_decode, for prompt processing (prefill speed, ds4 news
+ * summary, "speed benchmarks"); the permuted grouped form is this library's
+ * design. */
 ds4moe_status ds4moe_expert_ffn_grouped(const ds4moe_experts *ex, const void *x_bf16, int T, const int32_t *ids,
                                         const float *weights, int k, float *y_perm, int32_t *inv_perm,
                                         float *y_shared, void *ws, size_t ws_bytes, ds4moe_stream stream);
 
 /* out[t] = y_shared[t] + sum_{j<k} y_perm[inv_perm[t*k+j]] (j in increasing
- * order, fp32).  y_shared may be NULL.  d multiple of 4. */
+ * order, fp32).  y_shared may be NULL.  d multiple of 4.  This is the last
+ * line of the layer formula at the top of this file; the pages fix no
+ * summation order, so j runs in increasing order for a deterministic result. */
 ds4moe_status ds4moe_combine(const float *y_perm, const int32_t *inv_perm, const float *y_shared, int T, int d,
                              int k, float *out, ds4moe_stream stream);
 
