@@ -11,7 +11,9 @@ pass.  The timed region replays a CUDA graph of one step K times.
 
 Also reported: the dominant kernel's roofline (the gate/up GEMV, HBM-bound),
 an end-to-end number through the public Python API with host<->device copies,
-the CPU oracle as baseline, and a prefill measurement (T=4096, grouped GEMM).
+the CPU oracle as baseline, a prefill measurement (T=4096, grouped GEMM) and,
+on one GPU, the other workloads: the tiny latency case, the batched decode
+sweep (B = 1, 4, 16, 64) and the Q4K layer (T=16384 prefill, B=1 decode).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 Multi-GPU: data-parallel replicas (each rank decodes its own token stream);
@@ -56,6 +58,12 @@ def layer_bytes(wl):
     s = wl.shape
     routed = s.k * (2 * s.f * (s.d // 256) * 66 + s.d * (s.f // 256) * 84)
     return routed + s.shared_bytes + s.router_bytes + s.d * 2 + s.d * 4
+
+
+def step_bytes(shape, n_unique, B):
+    """Algorithmic bytes of one decode step of B tokens that touches n_unique distinct experts: each touched
+    expert's packed blocks once, the shared expert and router once, x in (bf16) and out (fp32)."""
+    return n_unique * shape.expert_bytes + shape.shared_bytes + shape.router_bytes + B * shape.d * (2 + 4)
 
 
 def gateup_bytes(wl):
@@ -334,6 +342,10 @@ def run_ours(args, ws, rank, local):
     if not args.no_prefill:
         prefill = run_prefill(args, ds4moe, torch, stream, tf, tf_sus, peak_kind)
 
+    workloads = None
+    if ws == 1 and not args.no_workloads:
+        workloads = run_workloads(ds4moe, torch, stream, hbm, tf, peak_kind)
+
     if rank != 0:
         return
     cpu = None
@@ -362,6 +374,7 @@ def run_ours(args, ws, rank, local):
                         "median of 3 runs of 256 tokens", "eager_forward_value": e2e_eager},
         "clocks": clk.summary(),
         "prefill": prefill,
+        "workloads": workloads,
         "setup_s": setup_s,
     }
     print(json.dumps(line), flush=True)
@@ -398,6 +411,133 @@ def run_prefill(args, ds4moe, torch, stream, tf, tf_sus, peak_kind):
     return {"workload": "prefill T=%d, same layer, router bias N(0,1)" % T, "tokens_per_s": T / (ms / 1e3),
             "ms_per_step": ms, "tflops": flops / (ms / 1e3) / 1e12,
             "frac_of_bf16_peak": flops / (ms / 1e3) / 1e12 / tf, "peak_tflops": tf, "peak_kind": peak_kind}
+
+
+class StepTimer:
+    """Device time of single steps with L2 flushed in between: each step is bracketed by CUDA events on the
+    stream, and a 1 GiB write (8x L2) runs between steps, outside the events.  The flush also keeps the GPU busy
+    long enough for the host to enqueue the next step ahead of it, so host launch time normally does not enter."""
+
+    def __init__(self, torch, stream):
+        self.torch, self.stream = torch, stream
+        self.flush = torch.empty(1 << 28, dtype=torch.float32, device="cuda")
+
+    def mean_ms(self, step, n, warmup=2):
+        torch, st = self.torch, self.stream
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+        torch.cuda.synchronize()
+        with torch.cuda.stream(st):
+            for i in range(warmup):
+                step(i)
+            self.flush.zero_()
+            self.flush.zero_()
+            for i in range(n):
+                ev[i][0].record(st)
+                step(i)
+                ev[i][1].record(st)
+                self.flush.zero_()
+            st.synchronize()
+        return float(np.mean([a.elapsed_time(b) for a, b in ev]))
+
+
+def run_workloads(ds4moe, torch, stream, hbm, tf, peak_kind):
+    """The other workloads of the layer, one GPU: the tiny latency case, the batched decode sweep (B = 1, 4, 16,
+    64 with skewed routing: distinct experts touched, bytes, GB/s) and the Q4K layer (T=16384 prefill, then B=1
+    decode).  Each runs the same entry points, at the same sizes, as the parity tests; a failure is reported in
+    its entry instead of the numbers."""
+    res = {}
+    timer = StepTimer(torch, stream)
+
+    def guarded(name, fn):
+        try:
+            res[name] = fn()
+        except Exception as exc:  # report, keep the main line
+            res[name] = {"error": "%s: %s" % (type(exc).__name__, str(exc)[:200])}
+
+    def tiny():
+        wl = synth.WORKLOADS["tiny"]
+        D = ds4moe.DeviceLayer(synth.make_layer(wl), max_tokens=1)
+        with torch.cuda.stream(stream):
+            G = D.decode_graph()
+            G(torch.from_numpy(synth.activations(wl, 1)).cuda())
+            n = 2000
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            for _ in range(20):
+                G()
+            e0.record(stream)
+            for _ in range(n):
+                G()
+            e1.record(stream)
+            stream.synchronize()
+        us = e0.elapsed_time(e1) * 1e3 / n
+        s = wl.shape
+        return {"workload": "tiny d=%d E=%d f=%d k=%d shared_f=%d B=1 (L2-resident: a latency case)"
+                            % (s.d, s.E, s.f, s.k, s.f_shared),
+                "us_per_token": us, "tokens_per_s": 1e6 / us, "bytes_per_token": step_bytes(s, s.k, 1),
+                "timing": "%d back-to-back DecodeGraph replays (route + gate/up + down), CUDA events" % n}
+
+    def batched():
+        wl = synth.WORKLOADS["batched"]
+        s = wl.shape
+        D = ds4moe.DeviceLayer(synth.make_layer(wl), max_tokens=max(wl.tokens))
+        n = 16
+        rows = []
+        for B in wl.tokens:
+            x = torch.from_numpy(synth.activations(wl, B * n, stream=40 + B)).cuda().view(torch.bfloat16)
+            ids = [None] * n
+
+            def step(i):
+                _, ids[i], _ = D.forward(x[i * B:(i + 1) * B], return_routing=True)
+
+            ms = timer.mean_ms(step, n)
+            assert ds4moe.last_device_error() == 0
+            U = [len(np.unique(t.cpu().numpy())) for t in ids]
+            nbytes = float(np.mean([step_bytes(s, u, B) for u in U]))
+            rows.append({"B": B, "tokens_per_s": B / (ms / 1e3), "ms_per_step": ms,
+                         "unique_experts_per_step": float(np.mean(U)), "bytes_per_step": nbytes,
+                         "GBps": nbytes / (ms / 1e3) / 1e9, "frac_of_hbm": nbytes / (ms / 1e3) / 1e9 / hbm})
+        return {"workload": "batched decode, decode layer with router bias N(0,1), B in %s" % (list(wl.tokens),),
+                "timing": "mean of %d steps (distinct tokens each), L2 flushed between steps" % n,
+                "peak_GBps": hbm, "peak_kind": peak_kind, "sweep": rows}
+
+    def q4():
+        wl = synth.WORKLOADS["q4"]
+        s = wl.shape
+        T = wl.tokens[0]
+        D = ds4moe.DeviceLayer(synth.make_layer(wl), max_tokens=T)
+        x = torch.from_numpy(synth.activations(wl, T)).cuda().view(torch.bfloat16)
+        with torch.cuda.stream(stream):
+            for _ in range(2):
+                D.forward_grouped(x)
+            stream.synchronize()
+            n = 5
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(n):
+                D.forward_grouped(x)
+            e1.record(stream)
+            stream.synchronize()
+        ms = e0.elapsed_time(e1) / n
+        flops = 2 * 3 * s.d * s.f * T * s.k + 2 * 3 * s.d * s.f_shared * T + 2 * T * s.E * s.d
+        prefill = {"T": T, "tokens_per_s": T / (ms / 1e3), "ms_per_step": ms, "tflops": flops / (ms / 1e3) / 1e12,
+                   "frac_of_bf16_peak": flops / (ms / 1e3) / 1e12 / tf}
+        del x
+        n = 32
+        x1 = torch.from_numpy(synth.activations(wl, n, stream=1)).cuda().view(torch.bfloat16)
+        ms1 = timer.mean_ms(lambda i: D.forward(x1[i:i + 1]), n)
+        assert ds4moe.last_device_error() == 0
+        nb = step_bytes(s, s.k, 1)
+        decode = {"B": 1, "tokens_per_s": 1e3 / ms1, "ms_per_token": ms1, "bytes_per_token": nb,
+                  "GBps": nb / (ms1 / 1e3) / 1e9, "frac_of_hbm": nb / (ms1 / 1e3) / 1e9 / hbm,
+                  "path": "grouped (no Q4K GEMV yet)", "timing": "mean of %d tokens, L2 flushed between" % n}
+        return {"workload": "q4: decode layer with Q4K gate/up/down, router bias N(0,1)", "prefill": prefill,
+                "decode": decode, "peak_kind": peak_kind}
+
+    guarded("tiny", tiny)
+    guarded("batched", batched)
+    guarded("q4", q4)
+    del timer
+    return res
 
 
 def run_profile_case(args):
@@ -438,6 +578,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true", help="skip the tiny / batched / q4 measurements")
     ap.add_argument("--profile-case", action="store_true", help="small case for ncu captures (see profiles/)")
     ap.add_argument("--profile-prefill", type=int, default=0, help="with --profile-case: also run a T-token prefill")
     args = ap.parse_args()

@@ -29,3 +29,18 @@ def test_algorithmic_bytes_of_the_decode_workload():
     # routed IQ2X gate + up (66 B / 256 weights) + shared bf16 gate + up + x (bf16)
     want = s.k * 2 * s.f * s.d // 256 * 66 + 2 * s.f_shared * s.d * 2 + s.d * 2
     assert bench.gateup_bytes(wl) == want == 68165632
+
+
+def test_step_bytes_counts_each_touched_expert_once():
+    from bit_quantized_moe_02_b200 import synth
+    s = synth.WORKLOADS["decode"].shape
+    q4 = synth.WORKLOADS["q4"].shape
+    # per expert: IQ2X gate and up [2048 x 4096] at 66 B per 256 weights, Q2K down [4096 x 2048] at 84 B
+    assert s.expert_bytes == 2 * 2048 * 16 * 66 + 4096 * 8 * 84 == 7077888
+    assert q4.expert_bytes == 3 * 2048 * 4096 // 256 * 144 == 14155776
+    fixed = s.shared_bytes + s.router_bytes
+    assert bench.step_bytes(s, 0, 0) == fixed == 3 * 2048 * 4096 * 2 + 256 * 4096 * 2
+    assert bench.step_bytes(s, 24, 4) - bench.step_bytes(s, 23, 4) == s.expert_bytes
+    assert bench.step_bytes(s, 24, 5) - bench.step_bytes(s, 24, 4) == 4096 * (2 + 4)
+    # the B = 1 decode workload touches k experts: the same bytes as the main line's per-token figure
+    assert bench.step_bytes(s, s.k, 1) == bench.layer_bytes(synth.WORKLOADS["decode"])
