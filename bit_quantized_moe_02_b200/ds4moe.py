@@ -2,7 +2,10 @@
 
 Tensors are torch CUDA tensors; every call runs on the current torch stream.
 Nothing here computes any part of the layer: each step runs in the library's
-kernels, and a missing library raises instead of falling back.
+kernels, and a missing library raises instead of falling back.  Each tensor
+argument is checked before the call (on the current CUDA device, contiguous,
+the element size and shape or size the call reads or writes), since the
+library itself sees only plain pointers.
 """
 from __future__ import annotations
 
@@ -87,6 +90,36 @@ def _p(t: Optional[torch.Tensor]):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
+def _arg(t: Optional[torch.Tensor], what: str, dev: int, esize: int, shape=None, numel: Optional[int] = None,
+         optional: bool = False):
+    """Pointer of a tensor argument after the checks the library cannot make on a plain pointer: a contiguous
+    tensor on the current CUDA device, of the element size and shape (or at least the element count) the call
+    reads or writes.  A host tensor or a short buffer raises here instead of reaching the kernels."""
+    if t is None:
+        if optional:
+            return None
+        raise ValueError("%s: a tensor is required" % what)
+    if not t.is_cuda or t.device.index != dev:
+        raise ValueError("%s: expected a tensor on the current CUDA device (cuda:%d), got %s" % (what, dev, t.device))
+    if not t.is_contiguous():
+        raise ValueError("%s: expected a contiguous tensor" % what)
+    if t.element_size() != esize:
+        raise ValueError("%s: expected %d-byte elements, got %s" % (what, esize, t.dtype))
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError("%s: expected shape %s, got %s" % (what, tuple(shape), tuple(t.shape)))
+    if numel is not None and t.numel() < numel:
+        raise ValueError("%s: expected at least %d elements, got %d" % (what, numel, t.numel()))
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _bytes(t: torch.Tensor) -> int:
+    return t.numel() * t.element_size()
+
+
+def _cur() -> int:
+    return torch.cuda.current_device()
+
+
 def _stream():
     return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
 
@@ -102,13 +135,20 @@ def prepare(fmt: str, canonical: torch.Tensor, rows: int, cols: int, n_mats: int
     stride = (prepared_bytes(fmt, rows, cols) + 255) // 256 * 256
     if out is None:
         out = torch.empty(stride * max(n_mats, 1), dtype=torch.uint8, device=canonical.device)
-    _check(lib().ds4moe_prepare(FMT[fmt], _p(canonical), _p(out), rows, cols, n_mats, stride, _stream()), "prepare")
+    dev = _cur()
+    nbytes = n_mats * rows * (cols // 256) * synth.BLOCK_BYTES.get(fmt, 0)
+    pc = _arg(canonical, "prepare: canonical", dev, 1, numel=nbytes)
+    po = _arg(out, "prepare: out", dev, 1, numel=stride * n_mats)
+    _check(lib().ds4moe_prepare(FMT[fmt], pc, po, rows, cols, n_mats, stride, _stream()), "prepare")
     return out
 
 
 def dequant(fmt: str, prepared: torch.Tensor, codebook: Optional[torch.Tensor], rows: int, cols: int) -> torch.Tensor:
     out = torch.empty((rows, cols), dtype=torch.float32, device=prepared.device)
-    _check(lib().ds4moe_dequant(FMT[fmt], _p(prepared), _p(codebook), rows, cols, _p(out), _stream()), "dequant")
+    dev = _cur()
+    pp = _arg(prepared, "dequant: prepared", dev, 1, numel=prepared_bytes(fmt, rows, cols))
+    pg = _arg(codebook, "dequant: codebook", dev, 1, numel=256 * 8, optional=fmt != "iq2x")
+    _check(lib().ds4moe_dequant(FMT[fmt], pp, pg, rows, cols, _p(out), _stream()), "dequant")
     return out
 
 
@@ -120,8 +160,14 @@ def route(x: torch.Tensor, wr: torch.Tensor, bias: Optional[torch.Tensor], k: in
         ws = torch.empty(max(int(lib().ds4moe_route_workspace_size(T, d, E)), 1), dtype=torch.uint8, device=x.device)
     ids = torch.empty((T, k), dtype=torch.int32, device=x.device) if ids is None else ids
     weights = torch.empty((T, k), dtype=torch.float32, device=x.device) if weights is None else weights
-    _check(lib().ds4moe_route(_p(x), T, d, _p(wr), _p(bias), E, k, _p(ids), _p(weights), _p(ws), ws.numel(),
-                              _stream()), "route")
+    dev = _cur()
+    px = _arg(x, "route: x", dev, 2)
+    pw = _arg(wr, "route: w_router", dev, 2, shape=(E, d))
+    pb = _arg(bias, "route: bias", dev, 4, shape=(E,), optional=True)
+    pi = _arg(ids, "route: ids", dev, 4, shape=(T, k))
+    pr = _arg(weights, "route: weights", dev, 4, shape=(T, k))
+    ps = _arg(ws, "route: workspace", dev, ws.element_size())
+    _check(lib().ds4moe_route(px, T, d, pw, pb, E, k, pi, pr, ps, _bytes(ws), _stream()), "route")
     return ids, weights
 
 
@@ -133,42 +179,75 @@ def expert_ffn_decode(ex: Experts, x: torch.Tensor, ids: torch.Tensor, weights: 
                       out: Optional[torch.Tensor] = None) -> torch.Tensor:
     B, k = ids.shape
     out = torch.empty((B, ex.d), dtype=torch.float32, device=x.device) if out is None else out
-    _check(lib().ds4moe_expert_ffn_decode(ctypes.byref(ex), _p(x), B, _p(ids), _p(weights), k, _p(out), _p(ws),
-                                          ws.numel(), _stream()), "expert_ffn_decode")
+    dev = _cur()
+    px = _arg(x, "expert_ffn_decode: x", dev, 2, shape=(B, ex.d))
+    pi = _arg(ids, "expert_ffn_decode: ids", dev, 4)
+    pr = _arg(weights, "expert_ffn_decode: weights", dev, 4, shape=(B, k))
+    po = _arg(out, "expert_ffn_decode: out", dev, 4, shape=(B, ex.d))
+    ps = _arg(ws, "expert_ffn_decode: workspace", dev, ws.element_size())
+    _check(lib().ds4moe_expert_ffn_decode(ctypes.byref(ex), px, B, pi, pr, k, po, ps, _bytes(ws), _stream()),
+           "expert_ffn_decode")
     return out
 
 
 def decode_gateup(ex: Experts, x: torch.Tensor, ids: torch.Tensor, ws: torch.Tensor) -> None:
-    _check(lib().ds4moe_decode_gateup(ctypes.byref(ex), _p(x), _p(ids), ids.shape[-1], _p(ws), ws.numel(), _stream()),
-           "decode_gateup")
+    k = ids.shape[-1]
+    dev = _cur()
+    px = _arg(x, "decode_gateup: x", dev, 2, numel=ex.d)
+    pi = _arg(ids, "decode_gateup: ids", dev, 4, numel=k)
+    ps = _arg(ws, "decode_gateup: workspace", dev, ws.element_size())
+    _check(lib().ds4moe_decode_gateup(ctypes.byref(ex), px, pi, k, ps, _bytes(ws), _stream()), "decode_gateup")
 
 
 def decode_down(ex: Experts, ids: torch.Tensor, weights: torch.Tensor, ws: torch.Tensor, out: torch.Tensor) -> None:
-    _check(lib().ds4moe_decode_down(ctypes.byref(ex), _p(ids), _p(weights), ids.shape[-1], _p(out), _p(ws),
-                                    ws.numel(), _stream()), "decode_down")
+    k = ids.shape[-1]
+    dev = _cur()
+    pi = _arg(ids, "decode_down: ids", dev, 4, numel=k)
+    pr = _arg(weights, "decode_down: weights", dev, 4, numel=k)
+    po = _arg(out, "decode_down: out", dev, 4, numel=ex.d)
+    ps = _arg(ws, "decode_down: workspace", dev, ws.element_size())
+    _check(lib().ds4moe_decode_down(ctypes.byref(ex), pi, pr, k, po, ps, _bytes(ws), _stream()), "decode_down")
 
 
 def expert_ffn_decode_noalloc(ex: Experts, x: torch.Tensor, ids: torch.Tensor, weights: torch.Tensor,
                               out: Optional[torch.Tensor] = None) -> torch.Tensor:
     """B = 1 decode served from the library's fixed scratch array (no workspace argument)."""
     out = torch.empty((1, ex.d), dtype=torch.float32, device=x.device) if out is None else out
-    _check(lib().ds4moe_expert_ffn_decode_noalloc(ctypes.byref(ex), _p(x), _p(ids), _p(weights), ids.shape[-1],
-                                                  _p(out), _stream()), "expert_ffn_decode_noalloc")
+    k = ids.shape[-1]
+    dev = _cur()
+    px = _arg(x, "expert_ffn_decode_noalloc: x", dev, 2, numel=ex.d)
+    pi = _arg(ids, "expert_ffn_decode_noalloc: ids", dev, 4, numel=k)
+    pr = _arg(weights, "expert_ffn_decode_noalloc: weights", dev, 4, numel=k)
+    po = _arg(out, "expert_ffn_decode_noalloc: out", dev, 4, numel=ex.d)
+    _check(lib().ds4moe_expert_ffn_decode_noalloc(ctypes.byref(ex), px, pi, pr, k, po, _stream()),
+           "expert_ffn_decode_noalloc")
     return out
 
 
 def expert_ffn_grouped(ex: Experts, x: torch.Tensor, ids: torch.Tensor, weights: torch.Tensor, ws: torch.Tensor,
                        y_perm: torch.Tensor, inv_perm: torch.Tensor, y_shared: Optional[torch.Tensor]) -> None:
     T, k = ids.shape
-    _check(lib().ds4moe_expert_ffn_grouped(ctypes.byref(ex), _p(x), T, _p(ids), _p(weights), k, _p(y_perm),
-                                           _p(inv_perm), _p(y_shared), _p(ws), ws.numel(), _stream()),
-           "expert_ffn_grouped")
+    dev = _cur()
+    px = _arg(x, "expert_ffn_grouped: x", dev, 2, shape=(T, ex.d))
+    pi = _arg(ids, "expert_ffn_grouped: ids", dev, 4)
+    pr = _arg(weights, "expert_ffn_grouped: weights", dev, 4, shape=(T, k))
+    py = _arg(y_perm, "expert_ffn_grouped: y_perm", dev, 4, numel=T * k * ex.d)
+    pv = _arg(inv_perm, "expert_ffn_grouped: inv_perm", dev, 4, numel=T * k)
+    pz = _arg(y_shared, "expert_ffn_grouped: y_shared", dev, 4, numel=T * ex.d, optional=True)
+    ps = _arg(ws, "expert_ffn_grouped: workspace", dev, ws.element_size())
+    _check(lib().ds4moe_expert_ffn_grouped(ctypes.byref(ex), px, T, pi, pr, k, py, pv, pz, ps, _bytes(ws),
+                                           _stream()), "expert_ffn_grouped")
 
 
 def combine(y_perm: torch.Tensor, inv_perm: torch.Tensor, y_shared: Optional[torch.Tensor], T: int, d: int, k: int,
             out: Optional[torch.Tensor] = None) -> torch.Tensor:
     out = torch.empty((T, d), dtype=torch.float32, device=y_perm.device) if out is None else out
-    _check(lib().ds4moe_combine(_p(y_perm), _p(inv_perm), _p(y_shared), T, d, k, _p(out), _stream()), "combine")
+    dev = _cur()
+    py = _arg(y_perm, "combine: y_perm", dev, 4, numel=T * k * d)
+    pv = _arg(inv_perm, "combine: inv_perm", dev, 4, numel=T * k)
+    pz = _arg(y_shared, "combine: y_shared", dev, 4, numel=T * d, optional=True)
+    po = _arg(out, "combine: out", dev, 4, numel=T * d)
+    _check(lib().ds4moe_combine(py, pv, pz, T, d, k, po, _stream()), "combine")
     return out
 
 
