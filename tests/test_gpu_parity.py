@@ -146,6 +146,15 @@ def test_mid_shapes_decode_and_grouped(ds4, d, f, fs, E, k):
     run_and_compare(ds4, L, x, "grouped")  # several token tiles, ragged tail
 
 
+@pytest.mark.parametrize("d,f,fs,E,k", [(2048, 512, 1024, 16, 4), (4096, 1024, 2048, 16, 8)])
+def test_decode_gemv_shapes(ds4, d, f, fs, E, k):
+    """Single-token decode at the model's d with smaller f and E: other lane-slice widths of both GEMV kernels."""
+    shape = synth.LayerShape(d=d, E=E, f=f, k=k, f_shared=fs)
+    L = layer_of(shape, 1.0, 41 + f)
+    x = synth.f32_to_bf16_bits(synth.rng(6, d, f).normal(size=(3, d)).astype(np.float32))
+    run_and_compare(ds4, L, x, "decode")
+
+
 def test_q4k_layer_small(ds4):
     shape = synth.LayerShape(d=512, E=8, f=768, k=2, f_shared=256, fmt_gate="q4k", fmt_up="q4k", fmt_down="q4k")
     L = layer_of(shape, 1.0, 77)
