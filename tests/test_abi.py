@@ -103,3 +103,20 @@ def test_decode_gemv_limits_checked_on_host():
     assert lib.ds4moe_decode_gateup(ctypes.byref(ex), fake, fake, 2, fake, need - 1, None) == 4
     assert lib.ds4moe_expert_ffn_decode_noalloc(ctypes.byref(experts(768, 512)), fake, fake, fake, 2, fake,
                                                 None) == 2
+
+
+def test_empty_inputs_are_no_ops():
+    """Zero tokens: every many-token entry point returns OK without touching its (absent) buffers."""
+    lib = ds4moe.lib()
+    ex = ds4moe.Experts(256, 512, 8, 0, 0, 0, 1, 1 << 20, 1 << 21, 1 << 22, 1 << 16, 1 << 16, 1 << 16, 1 << 23,
+                        None, None, None)
+    assert lib.ds4moe_route(None, 0, 256, None, None, 8, 2, None, None, None, 0, None) == 0
+    assert lib.ds4moe_expert_ffn_decode(ctypes.byref(ex), None, 0, None, None, 2, None, None, 0, None) == 0
+    assert lib.ds4moe_expert_ffn_grouped(ctypes.byref(ex), None, 0, None, None, 2, None, None, None, None, 0,
+                                         None) == 0
+    assert lib.ds4moe_combine(None, None, None, 0, 256, 2, None, None) == 0
+    # negative counts are errors, not no-ops
+    assert lib.ds4moe_expert_ffn_decode(ctypes.byref(ex), None, -1, None, None, 2, None, None, 0, None) == 1
+    assert lib.ds4moe_expert_ffn_grouped(ctypes.byref(ex), None, -1, None, None, 2, None, None, None, None, 0,
+                                         None) == 1
+    assert lib.ds4moe_combine(None, None, None, -1, 256, 2, None, None) == 1
