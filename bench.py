@@ -344,7 +344,10 @@ def run_ours(args, ws, rank, local):
 
     workloads = None
     if ws == 1 and not args.no_workloads:
-        workloads = run_workloads(ds4moe, torch, stream, hbm, tf, peak_kind)
+        try:
+            workloads = run_workloads(ds4moe, torch, stream, hbm, tf, peak_kind)
+        except Exception as exc:  # these are reported beside the main line, which is kept either way
+            workloads = {"error": "%s: %s" % (type(exc).__name__, str(exc)[:200])}
 
     if rank != 0:
         return
