@@ -36,3 +36,24 @@ def test_bf16_rounding_nearest_even():
     bits = synth.f32_to_bf16_bits(v)
     back = (bits.astype(np.uint32) << 16).view(np.float32)
     assert back.tolist() == [1.0, 1.0, 1.0 + 2 ** -7, -2.5]
+
+
+def _top8(L, x):
+    xf = (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    logits = xf @ L.wr.view(np.float16).astype(np.float64).T + L.bias
+    return np.argsort(-logits, axis=1, kind="stable")[:, :8]
+
+
+def test_routing_skew_of_the_skewed_workloads():
+    """The router bias N(0, 1) gives the skew the workloads describe: at T=4096 the busiest expert gets about 10x
+    the mean load, and a batch of B tokens touches far fewer than 8 B distinct experts."""
+    wl = synth.WORKLOADS["prefill"]
+    counts = np.bincount(_top8(synth.make_layer(wl), synth.activations(wl, 4096)).ravel(), minlength=256)
+    assert 10 <= counts.max() / counts.mean() <= 17
+    wl = synth.WORKLOADS["batched"]
+    L = synth.make_layer(wl)
+    unique = []
+    for B in (4, 16, 64):
+        ids = _top8(L, synth.activations(wl, 8 * B, stream=40 + B)).reshape(8, B * 8)
+        unique.append(np.mean([len(np.unique(r)) for r in ids]))
+    assert 8 < unique[0] < unique[1] < unique[2] < 0.5 * 8 * 64
