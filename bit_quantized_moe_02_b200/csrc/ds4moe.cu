@@ -9,7 +9,7 @@
 
 #include "common.cuh"
 #include "decode_gemv.cuh"
-#include "grouped_mma.cuh"
+#include "grouped_common.cuh"
 #include "grouped_tc.cuh"
 #include "permute.cuh"
 #include "prepare.cuh"
@@ -199,23 +199,11 @@ struct GroupedWs {
     uint64_t total_grouped, total_decode;
     int nblk, max_tiles;
 };
-// The tcgen05 kernels run the grouped GEMMs; DS4MOE_GROUPED=mma selects the warp-level mma.sync kernels
-// instead (same results within rounding; kept for A/B measurement).
-bool use_tc_grouped() {
-    static int v = -1;
-    if (v < 0) {
-        const char *e = getenv("DS4MOE_GROUPED");
-        v = (e && e[0] == 'm') ? 0 : 1;
-    }
-    return v == 1;
-}
-int grouped_tile_n() { return use_tc_grouped() ? tc::NT : TILE_N; }
-
 GroupedWs grouped_ws(const ds4moe_experts *ex, int T, int k) {
     GroupedWs w;
     const uint64_t N = uint64_t(T) * k;
     w.nblk = int((N + PERM_BLOCK - 1) / PERM_BLOCK);
-    w.max_tiles = int(ex->E + (N + 63) / 64);  // enough for 64- and 128-token tiles
+    w.max_tiles = int(ex->E + (N + 63) / 64);  // >= the sum over experts of ceil(count / NT)
     uint64_t o = 0;
     auto take = [&](uint64_t bytes) {
         uint64_t r = o;
@@ -233,7 +221,7 @@ GroupedWs grouped_ws(const ds4moe_experts *ex, int T, int k) {
     w.meta = take(16);
     w.perm_tok = take(N * 4);
     w.perm_w = take(N * 4);
-    w.x_perm = take(use_tc_grouped() ? N * ex->d * 2 : 0);
+    w.x_perm = take(N * ex->d * 2);
     w.h16 = take(N * ex->f * 2);
     w.hs = take(uint64_t(T) * (ex->f_shared > 0 ? ex->f_shared : 1) * 2);
     w.total_grouped = o;
@@ -253,9 +241,7 @@ template <int AFMT, bool GATEUP>
 ds4moe_status launch_grouped(const GroupedArgs &ga, int row_units, int col_tiles, const void *b_tma, uint64_t b_rows,
                              cudaStream_t st) {
     if (row_units <= 0 || col_tiles <= 0) return DS4MOE_OK;
-    bool tc_path = true;
-    if constexpr (!tc::is_dense<AFMT>()) tc_path = use_tc_grouped();
-    if (tc_path) {
+    {
         constexpr bool bf16 = AFMT == tc::FMT_BF16D;
         CUtensorMap tb, ta0 = {}, ta1 = {};
         if (!make_tile_map(&tb, b_tma, b_rows, uint64_t(ga.K), bf16)) return DS4MOE_ECUDA;
@@ -282,12 +268,6 @@ ds4moe_status launch_grouped(const GroupedArgs &ga, int row_units, int col_tiles
         constexpr int smem = tc::Cfg<AFMT, GATEUP>::SMEM;
         if (!set_smem(kern, smem)) return DS4MOE_ECUDA;
         kern<<<dim3(row_units / tc::M, col_tiles), tc::THREADS, smem, st>>>(ga, tb, ta0, ta1, p0, p1, p2, p3);
-    } else {
-        if constexpr (!tc::is_dense<AFMT>()) {
-            auto kern = grouped_mma_kernel<AFMT, GATEUP>;
-            if (!set_smem(kern, GM_SMEM)) return DS4MOE_ECUDA;
-            kern<<<dim3(GATEUP ? row_units / 64 : row_units / GM_M, col_tiles), GM_THREADS, GM_SMEM, st>>>(ga);
-        }
     }
     DS4_CHECK_LAUNCH();
     return DS4MOE_OK;
@@ -319,17 +299,15 @@ ds4moe_status run_grouped(const ds4moe_experts *ex, const void *x, int T, const 
     const size_t hist_smem = size_t(ex->E) * 4;
     perm_count_kernel<<<W.nblk, PERM_BLOCK, hist_smem, st>>>(ids, N, ex->E, blk);
     DS4_CHECK_LAUNCH();
-    const int tile_n = grouped_tile_n();
+    const int tile_n = tc::NT;
     perm_scan_kernel<<<1, 1024, 0, st>>>(blk, W.nblk, ex->E, tile_n, counts, offsets, tile_e, tile_pos0, tile_cnt,
                                          meta);
     DS4_CHECK_LAUNCH();
     perm_scatter_kernel<<<W.nblk, PERM_BLOCK, hist_smem, st>>>(ids, weights, N, k, ex->E, blk, perm_tok, perm_w,
                                                                inv_perm);
     DS4_CHECK_LAUNCH();
-    if (use_tc_grouped()) {
-        gather_rows_kernel<<<(N + 7) / 8, 256, 0, st>>>(x16, ex->d, perm_tok, N, x_perm);
-        DS4_CHECK_LAUNCH();
-    }
+    gather_rows_kernel<<<(N + 7) / 8, 256, 0, st>>>(x16, ex->d, perm_tok, N, x_perm);
+    DS4_CHECK_LAUNCH();
 
     // routed GEMM-1: gate/up -> h16
     GroupedArgs g1 = {};
@@ -356,21 +334,18 @@ ds4moe_status run_grouped(const ds4moe_experts *ex, const void *x, int T, const 
 
     if (ex->f_shared > 0) {
         const int ct = (T + tile_n - 1) / tile_n;
-        // Shared expert, a dense bf16 SwiGLU: on the tensor-core path A and the tokens both come by TMA as bf16
-        // (x as given, hs written as bf16); the warp-MMA path dequantizes A into fp16 against x16 / fp16 hs.
-        const bool dense = use_tc_grouped();
+        // Shared expert, a dense bf16 SwiGLU: A and the tokens both come by TMA as bf16 (x as given, hs written
+        // as bf16)
         GroupedArgs s1 = {};
         s1.a0 = static_cast<const uint8_t *>(ex->sh_gate); s1.a1 = static_cast<const uint8_t *>(ex->sh_up);
         s1.a_stride = 0; s1.rows = ex->f_shared; s1.K = ex->d;
-        s1.b_src = x16; s1.b_colscale = dense ? nullptr : xinv; s1.n_pos = T; s1.out = hs; s1.ldo = ex->f_shared;
-        s = dense ? launch_grouped<tc::FMT_BF16D, true>(s1, ex->f_shared, ct, xb, T, st)
-                  : launch_grouped<DS4MOE_FMT_BF16, true>(s1, ex->f_shared, ct, x16, T, st);
+        s1.b_src = x16; s1.b_colscale = nullptr; s1.n_pos = T; s1.out = hs; s1.ldo = ex->f_shared;
+        s = launch_grouped<tc::FMT_BF16D, true>(s1, ex->f_shared, ct, xb, T, st);
         if (s != DS4MOE_OK) return s;
         GroupedArgs s2 = {};
         s2.a0 = static_cast<const uint8_t *>(ex->sh_down); s2.a_stride = 0; s2.rows = ex->d; s2.K = ex->f_shared;
         s2.b_src = hs; s2.n_pos = T; s2.out = y_shared; s2.ldo = ex->d;
-        s = dense ? launch_grouped<tc::FMT_BF16D, false>(s2, ex->d, ct, hs, T, st)
-                  : launch_grouped<DS4MOE_FMT_BF16, false>(s2, ex->d, ct, hs, T, st);
+        s = launch_grouped<tc::FMT_BF16D, false>(s2, ex->d, ct, hs, T, st);
         if (s != DS4MOE_OK) return s;
     }
     return DS4MOE_OK;

@@ -31,7 +31,7 @@
 #include <cuda.h>
 
 #include "common.cuh"
-#include "grouped_mma.cuh"
+#include "grouped_common.cuh"
 
 namespace ds4 {
 namespace tc {
@@ -203,11 +203,8 @@ template <int AFMT, bool GATEUP>
 struct SPackCfg;
 template <> struct SPackCfg<DS4MOE_FMT_IQ2X, true> { static constexpr int SS = 4, NW = 18; };   // one super-block
 template <> struct SPackCfg<DS4MOE_FMT_Q4K, true> { static constexpr int SS = 2, NW = 20; };    // half super-block
-template <> struct SPackCfg<DS4MOE_FMT_BF16, true> { static constexpr int SS = 1, NW = 32; };
 template <> struct SPackCfg<DS4MOE_FMT_Q2K, false> { static constexpr int SS = 4, NW = 13; };
 template <> struct SPackCfg<DS4MOE_FMT_Q4K, false> { static constexpr int SS = 4, NW = 20; };
-template <> struct SPackCfg<DS4MOE_FMT_BF16, false> { static constexpr int SS = 1, NW = 16; };
-template <> struct SPackCfg<FMT_F16, false> { static constexpr int SS = 1, NW = 16; };
 
 template <int AFMT, bool GATEUP>
 struct SPack {
@@ -257,10 +254,8 @@ __device__ __forceinline__ void sp_load(SPack<AFMT, GATEUP> &pk, const uint8_t *
         const uint32_t *sc = reinterpret_cast<const uint32_t *>(mat + P.off[1] + b * 12);
         pk.w[16] = sc[0]; pk.w[17] = sc[1]; pk.w[18] = sc[2];
         pk.w[19] = ldg_nc_u32(mat + P.off[2] + b * 4);
-    } else {  // BF16 / F16 dense rows: one stage = 64 (GATEUP) or 32 (DOWN, half h) elements
-        const uint8_t *p = mat + (size_t(row) * K + size_t(ss) * BK + (GATEUP ? 0 : h * 32)) * 2;
-#pragma unroll
-        for (int i = 0; i < SPackCfg<AFMT, GATEUP>::NW / 4; i++) ld4(pk.w + 4 * i, p + 16 * i);
+    } else {
+        static_assert(AFMT == DS4MOE_FMT_IQ2X, "packed formats only: dense rows come by TMA");
     }
 }
 
@@ -344,15 +339,8 @@ __device__ __forceinline__ void sp_dequant(const SPack<AFMT, GATEUP> &pk, int h,
                 oo[4 + p] = half2_as_u32(__highs2half2(P[2 * p], P[2 * p + 1]));
             }
         }
-    } else if constexpr (AFMT == FMT_F16) {
-#pragma unroll
-        for (int i = 0; i < SPackCfg<AFMT, GATEUP>::NW / 4; i++)
-            o[i] = make_uint4(pk.w[4 * i], pk.w[4 * i + 1], pk.w[4 * i + 2], pk.w[4 * i + 3]);
-    } else {  // BF16
-#pragma unroll
-        for (int i = 0; i < SPackCfg<AFMT, GATEUP>::NW / 4; i++)
-            o[i] = make_uint4(bf16x2_to_f16x2(pk.w[4 * i], inf), bf16x2_to_f16x2(pk.w[4 * i + 1], inf),
-                              bf16x2_to_f16x2(pk.w[4 * i + 2], inf), bf16x2_to_f16x2(pk.w[4 * i + 3], inf));
+    } else {
+        static_assert(AFMT == DS4MOE_FMT_IQ2X, "packed formats only: dense rows come by TMA");
     }
 }
 

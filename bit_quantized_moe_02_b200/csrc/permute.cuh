@@ -13,7 +13,6 @@
 namespace ds4 {
 
 constexpr int PERM_BLOCK = 1024;
-constexpr int TILE_N = 64;  // tokens per tile of the mma.sync grouped kernel
 
 // x16[t] = fp16(x[t] * 2^e_t) with max|x16[t]| in [2^13, 2^14); xinv[t] = 2^-e_t.
 __global__ void __launch_bounds__(256) prep_x_kernel(const __nv_bfloat16 *__restrict__ x, int d,
