@@ -183,12 +183,15 @@ def test_batched_decode(ds4, B):
     run_and_compare(ds4, L, x, "batched")
 
 
-def test_bad_expert_id_sets_device_error(ds4):
-    wl = synth.WORKLOADS["tiny"]
+@pytest.mark.parametrize("shape", [synth.WORKLOADS["tiny"].shape,
+                                   synth.LayerShape(d=2048, E=16, f=512, k=4, f_shared=1024)])
+def test_bad_expert_id_sets_device_error(ds4, shape):
+    wl = synth.Workload("bad_id", shape, (1,), 0.0, 13)
     D = ds4.DeviceLayer(synth.make_layer(wl))
     x = dev(synth.activations(wl, 1)).view(torch.bfloat16)
-    ids = torch.tensor([[1, 99]], dtype=torch.int32, device="cuda")  # 99 >= E: skipped on the device, flagged
-    w = torch.tensor([[0.5, 0.5]], dtype=torch.float32, device="cuda")
+    bad = [1, 99] + list(range(2, shape.k))  # 99 >= E: skipped on the device, flagged
+    ids = torch.tensor([bad], dtype=torch.int32, device="cuda")
+    w = torch.full((1, shape.k), 1.0 / shape.k, dtype=torch.float32, device="cuda")
     ds4.expert_ffn_decode(D.ex, x, ids, w, D.ws)
     assert ds4.last_device_error() == 6
     assert ds4.last_device_error() == 0  # read clears
