@@ -5,6 +5,7 @@
 #include <stdio.h>
 #include <stdlib.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
@@ -133,6 +134,12 @@ bool make_plane_map(CUtensorMap *m, const void *base, uint64_t row_bytes, uint64
 
 bool fmt_quant(int f) { return f == DS4MOE_FMT_IQ2X || f == DS4MOE_FMT_Q2K || f == DS4MOE_FMT_Q4K; }
 
+// The permutation's offset scan (perm_scan_kernel) is one CTA of 1024 threads, one per expert: the grouped path
+// takes at most this many experts, and expert intermediate sizes f up to tc::MAX_K (the down GEMM keeps one
+// scale per 128-wide K range on chip).
+constexpr int MAX_E_GROUPED = 1024;
+bool grouped_supported(const ds4moe_experts *ex) { return ex->E <= MAX_E_GROUPED && ex->f <= tc::MAX_K; }
+
 ds4moe_status check_experts(const ds4moe_experts *ex) {
     if (!ex) return DS4MOE_EINVAL;
     if (ex->d <= 0 || ex->f <= 0 || ex->E <= 0 || ex->d % QK || ex->f % QK || ex->f_shared < 0 ||
@@ -194,7 +201,7 @@ DecodeWs decode_ws(const ds4moe_experts *ex, int k) {
 }
 
 struct GroupedWs {
-    uint64_t x16, xinv, blk, counts, offsets, tile_e, tile_pos0, tile_cnt, meta, perm_tok, perm_w, x_perm, h16, hs;
+    uint64_t x16, xinv, blk, counts, offsets, tile_e, tile_pos0, tile_cnt, meta, perm_tok, perm_w, x_perm, h16, hexp, hs;
     uint64_t y_perm, inv, y_shared;  // only used when decode B > 1 runs through the grouped path
     uint64_t total_grouped, total_decode;
     int nblk, max_tiles;
@@ -223,6 +230,7 @@ GroupedWs grouped_ws(const ds4moe_experts *ex, int T, int k) {
     w.perm_w = take(N * 4);
     w.x_perm = take(N * ex->d * 2);
     w.h16 = take(N * ex->f * 2);
+    w.hexp = take(uint64_t(w.max_tiles) * (ex->f / tc::M) * 4);  // fp16 h exponent per (token tile, row tile)
     w.hs = take(uint64_t(T) * (ex->f_shared > 0 ? ex->f_shared : 1) * 2);
     w.total_grouped = o;
     w.y_perm = take(N * ex->d * 4);
@@ -291,6 +299,7 @@ ds4moe_status run_grouped(const ds4moe_experts *ex, const void *x, int T, const 
     float *perm_w = reinterpret_cast<float *>(ws + W.perm_w);
     __half *x_perm = reinterpret_cast<__half *>(ws + W.x_perm);
     __half *h16 = reinterpret_cast<__half *>(ws + W.h16);
+    int32_t *hexp = reinterpret_cast<int32_t *>(ws + W.hexp);
     __half *hs = reinterpret_cast<__half *>(ws + W.hs);
     const __nv_bfloat16 *xb = static_cast<const __nv_bfloat16 *>(x);
 
@@ -316,7 +325,7 @@ ds4moe_status run_grouped(const ds4moe_experts *ex, const void *x, int T, const 
     g1.rows = ex->f; g1.K = ex->d; g1.codebook = ex->codebook;
     g1.b_src = x16; g1.b_rowidx = perm_tok; g1.b_colscale = xinv;
     g1.tile_e = tile_e; g1.tile_pos0 = tile_pos0; g1.tile_cnt = tile_cnt; g1.n_tiles = meta;
-    g1.out = h16; g1.ldo = ex->f;
+    g1.out = h16; g1.ldo = ex->f; g1.h_exp_out = hexp;
     ds4moe_status s;
     if (ex->fmt_gate == DS4MOE_FMT_IQ2X) s = launch_grouped<DS4MOE_FMT_IQ2X, true>(g1, ex->f, W.max_tiles, x_perm, N, st);
     else s = launch_grouped<DS4MOE_FMT_Q4K, true>(g1, ex->f, W.max_tiles, x_perm, N, st);
@@ -327,7 +336,7 @@ ds4moe_status run_grouped(const ds4moe_experts *ex, const void *x, int T, const 
     g2.a0 = D.down; g2.a_stride = D.down_stride; g2.pa = D.pd; g2.rows = ex->d; g2.K = ex->f; g2.n_mats = ex->E;
     g2.b_src = h16; g2.b_rowidx = nullptr; g2.b_colscale = nullptr;
     g2.tile_e = tile_e; g2.tile_pos0 = tile_pos0; g2.tile_cnt = tile_cnt; g2.n_tiles = meta;
-    g2.pos_weight = perm_w; g2.out = y_perm; g2.ldo = ex->d;
+    g2.pos_weight = perm_w; g2.out = y_perm; g2.ldo = ex->d; g2.h_exp_in = hexp;
     if (ex->fmt_down == DS4MOE_FMT_Q2K) s = launch_grouped<DS4MOE_FMT_Q2K, false>(g2, ex->d, W.max_tiles, h16, N, st);
     else s = launch_grouped<DS4MOE_FMT_Q4K, false>(g2, ex->d, W.max_tiles, h16, N, st);
     if (s != DS4MOE_OK) return s;
@@ -375,25 +384,28 @@ constexpr size_t NOALLOC_SCRATCH_BYTES = size_t(1) << 20;  // 1 MiB
 static __device__ __align__(256) uint8_t g_noalloc_scratch[NOALLOC_SCRATCH_BYTES];
 
 // Device address of g_noalloc_scratch per device.  The host-side symbol is only a stand-in, so the
-// address is looked up once per device, with that device current, and cached.
+// address is looked up once per device, with that device current, and cached.  Entries are atomics:
+// host threads making their first call on a device at the same time may both look the address up (the
+// same value), but never race on the entry.  A cached address does not survive cudaDeviceReset.
 void *noalloc_scratch_on_current_device(ds4moe_status *st) {
-    static void *cache[64] = {nullptr};
+    static std::atomic<void *> cache[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        (void)cudaGetLastError();
         *st = DS4MOE_ECUDA;
         return nullptr;
     }
-    if (!cache[dev]) {
-        void *p = nullptr;
+    void *p = cache[dev].load(std::memory_order_acquire);
+    if (!p) {
         if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
             (void)cudaGetLastError();
             *st = DS4MOE_ECUDA;
             return nullptr;
         }
-        cache[dev] = p;
+        cache[dev].store(p, std::memory_order_release);
     }
     *st = DS4MOE_OK;
-    return cache[dev];
+    return p;
 }
 
 }  // namespace
@@ -531,8 +543,10 @@ ds4moe_status ds4moe_route(const void *x_bf16, int T, int d, const void *w_route
 size_t ds4moe_workspace_size(const ds4moe_experts *ex, int T, int k) {
     if (check_experts(ex) != DS4MOE_OK || T < 0 || k < 1 || k > ex->E) return 0;
     const int TT = T > 0 ? T : 1;
+    const bool gemv = decode_gemv_supported(ex, k);
+    if (!grouped_supported(ex)) return TT == 1 && gemv ? decode_ws(ex, k).total : 0;  // no grouped path
     uint64_t need = grouped_ws(ex, TT, k).total_decode;
-    if (decode_gemv_supported(ex, k)) {
+    if (gemv) {
         const uint64_t dw = decode_ws(ex, k).total;
         if (dw > need) need = dw;
     }
@@ -558,6 +572,7 @@ ds4moe_status ds4moe_expert_ffn_decode(const ds4moe_experts *ex, const void *x_b
         return ds4moe_decode_down(ex, ids, weights, k, out, ws, ws_bytes, stream);
     }
     // B > 1 (or a format without a GEMV kernel): grouped path, then combine
+    if (!grouped_supported(ex)) return ex->E > MAX_E_GROUPED ? DS4MOE_EINVAL : DS4MOE_EUNSUPPORTED;
     const GroupedWs W = grouped_ws(ex, B, k);
     float *y_perm = reinterpret_cast<float *>(w8 + W.y_perm);
     int32_t *inv = reinterpret_cast<int32_t *>(w8 + W.inv);
@@ -648,7 +663,8 @@ ds4moe_status ds4moe_expert_ffn_grouped(const ds4moe_experts *ex, const void *x_
     (void)cudaGetLastError();  // report only errors raised by this call's launches
     ds4moe_status s = check_experts(ex);
     if (s != DS4MOE_OK) return s;
-    if (T < 0 || k < 1 || k > ex->E) return DS4MOE_EINVAL;
+    if (T < 0 || k < 1 || k > ex->E || ex->E > MAX_E_GROUPED) return DS4MOE_EINVAL;
+    if (!grouped_supported(ex)) return DS4MOE_EUNSUPPORTED;
     if (T == 0) return DS4MOE_OK;
     if (!x_bf16 || !ids || !weights || !y_perm || !inv_perm || !ws || !aligned16(x_bf16) || !aligned256(ws) ||
         !aligned16(y_perm))

@@ -26,6 +26,12 @@ struct GroupedArgs {
     const float *pos_weight;   // DOWN: factor per position, or NULL
     void *out;                 // GATEUP: [pos][rows] fp16;  DOWN: [pos][rows] fp32
     int ldo;
+    // Power-of-two exponents of the fp16 SwiGLU output, one per (token tile, 128-row tile of h): GATEUP writes
+    // h_exp_out[tile * (rows / 128) + row tile] = e >= 0 and stores h * 2^-e (e = 0 unless |h| > 65504); DOWN
+    // multiplies the weights of K range [128 i, 128 i + 128) by 2^h_exp_in[tile * (K / 128) + i], so each
+    // product, and the result, is unchanged.  NULL: no scaling.
+    int32_t *h_exp_out;
+    const int32_t *h_exp_in;
 };
 
 // 128-byte swizzle of a K-major fp16 tile: 16-byte chunk `chunk` of row `row`

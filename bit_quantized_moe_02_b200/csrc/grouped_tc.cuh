@@ -53,6 +53,7 @@ constexpr int A_TILE = M * BK * 2;   // 16 KB
 constexpr int B_TILE = NT * BK * 2;  // 16 KB
 constexpr int TABLE_BYTES = 256 * 8 * 16;
 constexpr long long WAIT_NS = 2000000000LL;  // 2 s bound on any single wait
+constexpr int MAX_K = 16384;                 // longest contraction of a packed DOWN operand (f)
 
 // Packed A planes streamed by TMA (3D maps: plane bytes x rows x experts) into a 2-slot shared-memory ring, one
 // slot per 256-wide K block of the tile's 128 rows: IQ2X gate/up (index and sign planes of both matrices, 16 KB)
@@ -274,9 +275,11 @@ __device__ __forceinline__ void q4k_pairs(uint32_t word, __half2 a2, __half2 c2,
 }
 
 // Dequantize stage j (compile-time) of a super-stage: GATEUP -> 8 uint4 (64 weights), DOWN -> 4 uint4 (32).
+// hsc: power-of-two factor on the DOWN weights (the inverse of the SwiGLU output's scale for this K range);
+// `inf` is raised when a scaled weight could leave the fp16 range.
 template <int AFMT, bool GATEUP, int J>
 __device__ __forceinline__ void sp_dequant(const SPack<AFMT, GATEUP> &pk, int h, int ss, const uint8_t *tbl_lane,
-                                           uint4 *o, bool &inf) {
+                                           uint4 *o, bool &inf, float hsc = 1.f) {
     constexpr uint32_t M = 0x80008000u;
     if constexpr (AFMT == DS4MOE_FMT_IQ2X) {
         const float dv = half_bits_to_float(uint16_t(pk.w[17]));
@@ -310,8 +313,14 @@ __device__ __forceinline__ void sp_dequant(const SPack<AFMT, GATEUP> &pk, int h,
             const int sub = GATEUP ? ((ss & 1) * 4 + 2 * J + u) : (2 * J + h);
             const int sc = q4k_field(pk.w[16], pk.w[17], pk.w[18], 6 * sub);
             const int mn = q4k_field(pk.w[16], pk.w[17], pk.w[18], 48 + 6 * sub);
-            const __half2 a2 = __float2half2_rn(dv * float(sc));
-            const __half2 c2 = __float2half2_rn(-(dm * float(mn)));
+            float av = dv * float(sc), cv = dm * float(mn);
+            if constexpr (!GATEUP) {
+                av *= hsc;
+                cv *= hsc;
+                inf |= !(fmaf(15.f, av, cv) <= 65504.f);
+            }
+            const __half2 a2 = __float2half2_rn(av);
+            const __half2 c2 = __float2half2_rn(-cv);
             const uint32_t *q = pk.w + (GATEUP ? (2 * J + u) * 4 : J * 4);
 #pragma unroll
             for (int w = 0; w < 4; w++) q4k_pairs(q[w], a2, c2, o[u * 4 + w]);
@@ -324,8 +333,10 @@ __device__ __forceinline__ void sp_dequant(const SPack<AFMT, GATEUP> &pk, int h,
 #pragma unroll
         for (int sb = 0; sb < 2; sb++) {
             const uint32_t scb = (scw >> (8 * sb)) & 0xFFu;
-            const __half2 a2 = __float2half2_rn(dv * float(scb & 15u));
-            const __half2 c2 = __float2half2_rn(-(dm * float(scb >> 4)));
+            const float av = dv * float(scb & 15u) * hsc, cv = dm * float(scb >> 4) * hsc;
+            inf |= !(fmaf(3.f, av, cv) <= 65504.f);
+            const __half2 a2 = __float2half2_rn(av);
+            const __half2 c2 = __float2half2_rn(-cv);
             __half2 P[8];
 #pragma unroll
             for (int p = 0; p < 8; p++) {
@@ -363,6 +374,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
     __shared__ float s_colsc[NT];
+    __shared__ uint32_t s_hmax;     // GATEUP: largest |h| of the tile (float bits; non-finite sorts above +inf)
+    __shared__ float s_hsc[MAX_K / 128];  // DOWN: weight factor 2^e of each 128-wide K range
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
@@ -400,8 +413,11 @@ __global__ void __launch_bounds__(THREADS, 1)
             mbar_init(empty_p(s), N_WA);
         }
         s_abort = 0;
+        s_hmax = 0;
         fence_mbar_init();
     }
+    if (!GATEUP && !DENSE && tid < a.K / 128)
+        s_hsc[tid] = a.h_exp_in ? ldexpf(1.f, a.h_exp_in[int(blockIdx.y) * (a.K / 128) + tid]) : 1.f;
     if (warp == 0) {
         tmem_alloc(smem_u32(&s_tmem), C::TMEM_COLS);
         tc_fence_before();
@@ -576,10 +592,11 @@ __global__ void __launch_bounds__(THREADS, 1)
                         break;
                     }
                     uint4 o[NOUT];
-                    if (jj == 0) sp_dequant<AFMT, GATEUP, 0>(cur, h, ss, tbl_lane, o, inf);
-                    else if (jj == 1) sp_dequant<AFMT, GATEUP, 1>(cur, h, ss, tbl_lane, o, inf);
-                    else if (jj == 2) sp_dequant<AFMT, GATEUP, 2>(cur, h, ss, tbl_lane, o, inf);
-                    else sp_dequant<AFMT, GATEUP, 3>(cur, h, ss, tbl_lane, o, inf);
+                    const float hsc = GATEUP ? 1.f : s_hsc[kc >> 1];
+                    if (jj == 0) sp_dequant<AFMT, GATEUP, 0>(cur, h, ss, tbl_lane, o, inf, hsc);
+                    else if (jj == 1) sp_dequant<AFMT, GATEUP, 1>(cur, h, ss, tbl_lane, o, inf, hsc);
+                    else if (jj == 2) sp_dequant<AFMT, GATEUP, 2>(cur, h, ss, tbl_lane, o, inf, hsc);
+                    else sp_dequant<AFMT, GATEUP, 3>(cur, h, ss, tbl_lane, o, inf, hsc);
                     uint8_t *ast = smem + s * C::STAGE + m * A_TILE;
 #pragma unroll
                     for (int c = 0; c < NOUT; c++)
@@ -627,10 +644,11 @@ __global__ void __launch_bounds__(THREADS, 1)
                         }
                         uint4 o[NOUT];
                         if constexpr (SS == 4) {
-                            if (jj == 0) sp_dequant<AFMT, GATEUP, 0>(cur, h, ss, tbl_lane, o, inf);
-                            else if (jj == 1) sp_dequant<AFMT, GATEUP, 1>(cur, h, ss, tbl_lane, o, inf);
-                            else if (jj == 2) sp_dequant<AFMT, GATEUP, 2>(cur, h, ss, tbl_lane, o, inf);
-                            else sp_dequant<AFMT, GATEUP, 3>(cur, h, ss, tbl_lane, o, inf);
+                            const float hsc = GATEUP ? 1.f : s_hsc[kc >> 1];
+                            if (jj == 0) sp_dequant<AFMT, GATEUP, 0>(cur, h, ss, tbl_lane, o, inf, hsc);
+                            else if (jj == 1) sp_dequant<AFMT, GATEUP, 1>(cur, h, ss, tbl_lane, o, inf, hsc);
+                            else if (jj == 2) sp_dequant<AFMT, GATEUP, 2>(cur, h, ss, tbl_lane, o, inf, hsc);
+                            else sp_dequant<AFMT, GATEUP, 3>(cur, h, ss, tbl_lane, o, inf, hsc);
                         } else if constexpr (SS == 2) {
                             if (jj == 0) sp_dequant<AFMT, GATEUP, 0>(cur, h, ss, tbl_lane, o, inf);
                             else sp_dequant<AFMT, GATEUP, 1>(cur, h, ss, tbl_lane, o, inf);
@@ -656,15 +674,18 @@ __global__ void __launch_bounds__(THREADS, 1)
             const int r = q * 32 + lane;
             const bool ok = __all_sync(0xffffffffu, mbar_wait(accum_bar, 0, abort_flag) && !*abort_flag);
             tc_fence_after();
-            if (ok) {
-                const uint32_t tq = tmem + (uint32_t(q * 32) << 16);
-                for (int c0 = 0; c0 < n_eff; c0 += 32) {
-                    uint32_t g[32];
-                    tmem_ld32(tq + c0, g);
-                    if constexpr (GATEUP) {
-                        uint32_t u[32];
+            const uint32_t tq = tmem + (uint32_t(q * 32) << 16);
+            if constexpr (GATEUP) {
+                // h = silu(g) * u of the tile's rows and tokens.  fp16 h is stored as h * 2^-e with one e >= 0
+                // per tile: e = 0 unless the tile's largest |h| exceeds the fp16 range, in which case the tile is
+                // written again with max |h| * 2^-e in [2^14, 2^15) (bf16 output for the dense shared expert
+                // needs no scale).  The down GEMM multiplies this K range of its weights by 2^e.
+                constexpr bool F16OUT = AFMT != FMT_BF16D;
+                auto store_pass = [&](float osc, uint32_t &amax_bits) {
+                    for (int c0 = 0; c0 < n_eff; c0 += 32) {
+                        uint32_t g[32], u[32];
+                        tmem_ld32(tq + c0, g);
                         tmem_ld32(tq + NT + c0, u);
-                        bool overflow = false;
 #pragma unroll
                         for (int i = 0; i < 32; i++) {
                             const int n = c0 + i;
@@ -672,19 +693,37 @@ __global__ void __launch_bounds__(THREADS, 1)
                                 const float sc = s_colsc[n];
                                 const float gv = __uint_as_float(g[i]) * sc, uv = __uint_as_float(u[i]) * sc;
                                 const float hv = silu(gv) * uv;
+                                amax_bits = max(amax_bits, __float_as_uint(hv) & 0x7FFFFFFFu);
                                 const size_t o = size_t(pos0 + n) * a.ldo + blockIdx.x * M + r;
-                                if constexpr (AFMT == FMT_BF16D) {
-                                    overflow |= !isfinite(hv);
-                                    reinterpret_cast<__nv_bfloat16 *>(a.out)[o] = __float2bfloat16_rn(hv);
-                                } else {
-                                    overflow |= !(fabsf(hv) <= 65504.f);
-                                    reinterpret_cast<__half *>(a.out)[o] = __float2half(hv);
-                                }
+                                if constexpr (F16OUT) reinterpret_cast<__half *>(a.out)[o] = __float2half(hv * osc);
+                                else reinterpret_cast<__nv_bfloat16 *>(a.out)[o] = __float2bfloat16_rn(hv);
                             }
                         }
-                        if (overflow) set_device_error(DS4MOE_EDEVICE);
-                    } else {
-                        float *out = reinterpret_cast<float *>(a.out);
+                    }
+                };
+                uint32_t amax_bits = 0;  // |h| as float bits: NaN sorts above +inf
+                if (ok) store_pass(1.f, amax_bits);
+                amax_bits = __reduce_max_sync(0xffffffffu, amax_bits);
+                if (lane == 0) atomicMax(&s_hmax, amax_bits);
+                asm volatile("bar.sync 1, 128;" ::: "memory");  // the four epilogue warps
+                const uint32_t tmax = *reinterpret_cast<volatile uint32_t *>(&s_hmax);
+                int he = 0;
+                if (tmax >= 0x7F800000u) {
+                    if (ok && r == 0) set_device_error(DS4MOE_EDEVICE);  // inf / NaN in the tile
+                } else if (F16OUT && tmax > 0x477FE000u) {                 // beyond 65504
+                    int qe;
+                    frexpf(__uint_as_float(tmax), &qe);
+                    he = qe - 15;
+                    uint32_t unused = 0;
+                    if (ok) store_pass(ldexpf(1.f, -he), unused);
+                }
+                if (ok && r == 0 && a.h_exp_out) a.h_exp_out[int(blockIdx.y) * gridDim.x + blockIdx.x] = he;
+            } else {
+                if (ok) {
+                    float *out = reinterpret_cast<float *>(a.out);
+                    for (int c0 = 0; c0 < n_eff; c0 += 32) {
+                        uint32_t g[32];
+                        tmem_ld32(tq + c0, g);
 #pragma unroll
                         for (int i = 0; i < 32; i++) {
                             const int n = c0 + i;

@@ -26,10 +26,23 @@
  *    (shapes, null pointers, 16-byte alignment, formats) return
  *    DS4MOE_EINVAL / DS4MOE_EUNSUPPORTED before anything is launched; a failed
  *    launch returns DS4MOE_ECUDA.
- *  - Data errors found on the device (an expert id outside [0, E), an
- *    activation that overflows fp16 inside the kernels, a bounded wait that
- *    ran out) do not trap: they set a per-device error word that
- *    ds4moe_last_device_error() reads and clears.
+ *  - Data errors found on the device do not trap: they set a per-device
+ *    error word that ds4moe_last_device_error() reads and clears.  What each
+ *    kernel checks:
+ *      DS4MOE_EDEVICE  an expert id outside [0, E): the decode gate/up and
+ *                      down kernels (that expert's rows are skipped) and the
+ *                      permutation of the grouped path (the pair is dropped);
+ *                      a non-finite SwiGLU output, or a scaled weight that
+ *                      would leave the fp16 range, in the grouped path's
+ *                      tensor-core kernels (see ds4moe_expert_ffn_grouped);
+ *      DS4MOE_ETIMEOUT a bounded wait (2 s) that ran out in the grouped
+ *                      path's tensor-core kernels (producer/consumer
+ *                      mbarrier pipeline).
+ *    The decode kernels need no fp16 range check: their fp16 sums are
+ *    bounded for any finite input (activations are scaled per token by a
+ *    power of two so that max |x| lies in [32, 64); an fp16 lane adds at
+ *    most 16 products of a codebook value <= 43 and |x| < 64, i.e. less than
+ *    44,032, or 4 products of q <= 3 and |h| < 64).
  *  - Matrices are [out x in], row-major; quantization blocks of 256 weights
  *    run along the input (contraction) dimension, so d and f are multiples of
  *    256.  Activations x are bf16 [T x d]; the layer output is fp32 [T x d]
@@ -157,22 +170,30 @@ ds4moe_status ds4moe_dequant(ds4moe_fmt fmt, const void *prepared, const uint8_t
  * with DS4MOE_ENOWORKSPACE.  Passage: the router is one of the parts left
  * unquantized (ds4 news summary, "model weights"); the pages do not give its
  * function, and this library reads it as the sigmoid -> top-k -> renormalise
- * rule written at the top of this file. */
+ * rule written at the top of this file.
+ * ds4moe_route_workspace_size: bytes of the router's workspace for T tokens (a
+ * library detail with no counterpart in the pages; 0 for invalid sizes). */
 size_t ds4moe_route_workspace_size(int T, int d, int E);
 ds4moe_status ds4moe_route(const void *x_bf16, int T, int d, const void *w_router_f16, const float *bias, int E,
                            int k, int32_t *ids, float *weights, void *ws, size_t ws_bytes, ds4moe_stream stream);
 
 /* Workspace for ds4moe_expert_ffn_decode / ds4moe_expert_ffn_grouped with T
- * tokens (B for decode) and top-k.  Alignment: 256 bytes. */
+ * tokens (B for decode) and top-k.  Alignment: 256 bytes.  Returns 0 when the
+ * layer or sizes are invalid, or when the call would need the grouped path
+ * and the layer is beyond its limits (E > 1024 or f > 16384).  A library
+ * detail with no counterpart in the pages (the pages describe no library
+ * interface). */
 size_t ds4moe_workspace_size(const ds4moe_experts *ex, int T, int k);
 
 /* Decode: out[B x d] (fp32) = the full layer output for B tokens, given the
  * routing (ids, weights) from ds4moe_route.  B = 1 runs the GEMV path (each
  * selected expert's packed rows streamed once and dequantized on the fly,
  * gate/up fused with SwiGLU, down fused with the weighted combine and the
- * shared expert) when the layer is IQ2X gate/up with Q2K down, d <= 8192 and
- * k <= 32; B > 1, and every other single-token layer, run the grouped path
- * internally (each touched expert read once).  On the GEMV path x_bf16 is read
+ * shared expert) when the layer is IQ2X gate/up with Q2K down, d and f are
+ * 256 times a power of two with d <= 8192 and f <= 8192, k <= 32 and the
+ * down kernel's staging of h fits in shared memory; B > 1, and every other
+ * single-token layer, run the grouped path internally (each touched expert
+ * read once; E <= 1024, else DS4MOE_EINVAL).  On the GEMV path x_bf16 is read
  * before the wait on the preceding kernel (see ds4moe_decode_gateup), so x
  * must not be written by the kernel launched just before this call on the
  * same stream; ds4moe_route between the two satisfies this.  Passage: the
@@ -187,7 +208,9 @@ ds4moe_status ds4moe_expert_ffn_decode(const ds4moe_experts *ex, const void *x_b
 /* The two launches of ds4moe_expert_ffn_decode's single-token GEMV path,
  * exposed so a caller can place other work or timing events between them
  * (B = 1; same layer limits as that path; same experts, workspace and stream
- * for both).  ds4moe_decode_gateup streams the k selected experts' gate/up
+ * for both).  Passage: the same expert FFN as ds4moe_expert_ffn_decode (ds4
+ * news summary, "model weights"); the split into two launches is this
+ * library's, with no counterpart in the pages.  ds4moe_decode_gateup streams the k selected experts' gate/up
  * rows and the shared expert's gate/up rows and leaves h_j = silu(G_j x) *
  * (U_j x) (fp32, k x f) and the shared expert's hs (fp32, f_shared) at the
  * start of the workspace; ds4moe_decode_down reads them and writes
@@ -212,10 +235,12 @@ ds4moe_status ds4moe_decode_down(const ds4moe_experts *ex, const int32_t *ids, c
  * limits are rejected with DS4MOE_EUNSUPPORTED, and a layer whose decode
  * scratch (4 * (k*f + f_shared) bytes, each part rounded up to 256) exceeds
  * 1 MiB with DS4MOE_ENOWORKSPACE (under the present limits every supported
- * layer fits).  Nothing is allocated: no cudaMalloc, no
+ * layer fits: the down kernel stages all k experts' h and the shared
+ * expert's in shared memory, which bounds the scratch far below 1 MiB).  Nothing is allocated: no cudaMalloc, no
  * cudaFree.  The first call on a device looks up the array's device address
- * (once per device, with that device current); make that first call before
- * any stream capture.  All calls share the one array, which keeps the last
+ * (once per device, with that device current) and caches it; make that
+ * first call before any stream capture.  The cached address does not survive
+ * cudaDeviceReset: do not use this entry point again after a reset.  All calls share the one array, which keeps the last
  * call's contents: calls whose kernels overlap on the GPU (other streams,
  * other threads) race on it, so serialize them. */
 ds4moe_status ds4moe_expert_ffn_decode_noalloc(const ds4moe_experts *ex, const void *x_bf16, const int32_t *ids,
@@ -229,10 +254,16 @@ ds4moe_status ds4moe_expert_ffn_decode_noalloc(const ds4moe_experts *ex, const v
  *   inv_perm int32 [T*k]:   inv_perm[t*k + j] = p,
  *   y_shared fp32 [T x d]:  the shared expert's output (may be NULL iff the
  *           layer has no shared expert).
- * Follow with ds4moe_combine.  Passage: the same expert FFN as
- * ds4moe_expert_ffn_decode, for prompt processing (prefill speed, ds4 news
- * summary, "speed benchmarks"); the permuted grouped form is this library's
- * design. */
+ * Follow with ds4moe_combine.  Limits: E <= 1024 (DS4MOE_EINVAL beyond),
+ * f <= 16384 (DS4MOE_EUNSUPPORTED beyond).  The SwiGLU output between the
+ * two expert GEMMs is kept in fp16 scaled by a power of two per 128-token
+ * tile and 128-row block (1 unless the block's largest |h| exceeds 65,504),
+ * and the down GEMM multiplies that block's weights back, so a large h is
+ * computed exactly as a small one; DS4MOE_EDEVICE is set only for a
+ * non-finite h or a scaled weight beyond the fp16 range.  Passage: the same
+ * expert FFN as ds4moe_expert_ffn_decode, for prompt processing (prefill
+ * speed, ds4 news summary, "speed benchmarks"); the permuted grouped form is
+ * this library's design. */
 ds4moe_status ds4moe_expert_ffn_grouped(const ds4moe_experts *ex, const void *x_bf16, int T, const int32_t *ids,
                                         const float *weights, int k, float *y_perm, int32_t *inv_perm,
                                         float *y_shared, void *ws, size_t ws_bytes, ds4moe_stream stream);

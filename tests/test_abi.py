@@ -80,9 +80,9 @@ def test_host_side_argument_checks():
 
 
 def test_decode_gemv_limits_checked_on_host():
-    """The single-token GEMV halves refuse layers outside their limits before any launch: d must be 256 times a
-    power of two up to 8192, f likewise, gate/up IQ2X with Q2K down, k <= 32; the combined decode call then
-    runs the grouped path instead (its own checks)."""
+    """The single-token GEMV halves refuse layers outside their limits before any launch: d and f 256 times a power
+    of two up to 8192, gate/up IQ2X with Q2K down, k <= 32; the combined decode call then runs the grouped path
+    instead (its own checks)."""
     lib = ds4moe.lib()
     fake = ctypes.c_void_p(1 << 20)
 
@@ -103,6 +103,26 @@ def test_decode_gemv_limits_checked_on_host():
     assert lib.ds4moe_decode_gateup(ctypes.byref(ex), fake, fake, 2, fake, need - 1, None) == 4
     assert lib.ds4moe_expert_ffn_decode_noalloc(ctypes.byref(experts(768, 512)), fake, fake, fake, 2, fake,
                                                 None) == 2
+
+
+def test_grouped_path_expert_limit():
+    """The grouped path's offset scan is one CTA of 1024 threads: more than 1024 experts are refused before any
+    launch (and the workspace query returns 0), while the single-token GEMV path, which has no such scan, still
+    takes such a layer."""
+    lib = ds4moe.lib()
+    fake = ctypes.c_void_p(1 << 20)
+    big = ds4moe.Experts(256, 512, 2048, 0, 0, 0, 1, 1 << 20, 1 << 21, 1 << 22, 1 << 16, 1 << 16, 1 << 16, 1 << 23,
+                         None, None, None)
+    assert lib.ds4moe_workspace_size(ctypes.byref(big), 4, 2) == 0
+    assert lib.ds4moe_workspace_size(ctypes.byref(big), 1, 2) > 0  # B = 1: GEMV path
+    assert lib.ds4moe_expert_ffn_grouped(ctypes.byref(big), fake, 4, fake, fake, 2, fake, fake, None, fake,
+                                         1 << 30, None) == 1
+    assert lib.ds4moe_expert_ffn_decode(ctypes.byref(big), fake, 4, fake, fake, 2, fake, fake, 1 << 30, None) == 1
+    q4big = ds4moe.Experts(256, 512, 2048, 0, 2, 2, 2, 1 << 20, 1 << 21, 1 << 22, 1 << 17, 1 << 17, 1 << 17, None,
+                           None, None, None)
+    assert lib.ds4moe_workspace_size(ctypes.byref(q4big), 1, 2) == 0  # Q4K B = 1 runs the grouped path
+    assert lib.ds4moe_expert_ffn_decode(ctypes.byref(q4big), fake, 1, fake, fake, 2, fake, fake, 1 << 30,
+                                        None) == 1
 
 
 def test_empty_inputs_are_no_ops():
