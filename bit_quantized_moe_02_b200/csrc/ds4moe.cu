@@ -189,6 +189,10 @@ bool decode_gemv_supported(const ds4moe_experts *ex, int k) {
     return dd_layout(k, ex->f, ex->f_shared).total <= 200 * 1024;
 }
 
+// Decode batches of up to this many tokens run the single-token GEMV pair once per token (each pass streams its
+// token's experts at the GEMV path's rate; see ds4moe_expert_ffn_decode), larger ones the grouped path.
+constexpr int DECODE_GEMV_MAX_B = 16;
+
 struct DecodeWs {
     uint64_t h, hs, total;  // h_j = silu(G_j x) * (U_j x) for the k experts [k x f]; shared expert's h [f_shared]
 };
@@ -544,13 +548,11 @@ size_t ds4moe_workspace_size(const ds4moe_experts *ex, int T, int k) {
     if (check_experts(ex) != DS4MOE_OK || T < 0 || k < 1 || k > ex->E) return 0;
     const int TT = T > 0 ? T : 1;
     const bool gemv = decode_gemv_supported(ex, k);
-    if (!grouped_supported(ex)) return TT == 1 && gemv ? decode_ws(ex, k).total : 0;  // no grouped path
+    // the GEMV path gives each token of a decode batch its own h region
+    const uint64_t gemv_need = gemv && TT <= DECODE_GEMV_MAX_B ? uint64_t(TT) * decode_ws(ex, k).total : 0;
+    if (!grouped_supported(ex)) return gemv_need;  // no grouped path: only the GEMV path's batches
     uint64_t need = grouped_ws(ex, TT, k).total_decode;
-    if (gemv) {
-        const uint64_t dw = decode_ws(ex, k).total;
-        if (dw > need) need = dw;
-    }
-    return need;
+    return need > gemv_need ? need : gemv_need;
 }
 
 ds4moe_status ds4moe_expert_ffn_decode(const ds4moe_experts *ex, const void *x_bf16, int B, const int32_t *ids,
@@ -566,10 +568,19 @@ ds4moe_status ds4moe_expert_ffn_decode(const ds4moe_experts *ex, const void *x_b
     if (ws_bytes < ds4moe_workspace_size(ex, B, k)) return DS4MOE_ENOWORKSPACE;
     cudaStream_t st = cs(stream);
     uint8_t *w8 = static_cast<uint8_t *>(ws);
-    if (B == 1 && decode_gemv_supported(ex, k)) {
-        s = ds4moe_decode_gateup(ex, x_bf16, ids, k, ws, ws_bytes, stream);
-        if (s != DS4MOE_OK) return s;
-        return ds4moe_decode_down(ex, ids, weights, k, out, ws, ws_bytes, stream);
+    if (B <= DECODE_GEMV_MAX_B && decode_gemv_supported(ex, k)) {
+        // token by token through the GEMV pair, each token with its own h region (256-byte aligned slices)
+        const uint64_t per = decode_ws(ex, k).total;
+        for (int t = 0; t < B; t++) {
+            uint8_t *wt = w8 + uint64_t(t) * per;
+            const void *xt = static_cast<const uint8_t *>(x_bf16) + size_t(t) * ex->d * 2;
+            s = ds4moe_decode_gateup(ex, xt, ids + size_t(t) * k, k, wt, per, stream);
+            if (s != DS4MOE_OK) return s;
+            s = ds4moe_decode_down(ex, ids + size_t(t) * k, weights + size_t(t) * k, k, out + size_t(t) * ex->d, wt, per,
+                                   stream);
+            if (s != DS4MOE_OK) return s;
+        }
+        return DS4MOE_OK;
     }
     // B > 1 (or a format without a GEMV kernel): grouped path, then combine
     if (!grouped_supported(ex)) return ex->E > MAX_E_GROUPED ? DS4MOE_EINVAL : DS4MOE_EUNSUPPORTED;

@@ -186,20 +186,26 @@ ds4moe_status ds4moe_route(const void *x_bf16, int T, int d, const void *w_route
 size_t ds4moe_workspace_size(const ds4moe_experts *ex, int T, int k);
 
 /* Decode: out[B x d] (fp32) = the full layer output for B tokens, given the
- * routing (ids, weights) from ds4moe_route.  B = 1 runs the GEMV path (each
- * selected expert's packed rows streamed once and dequantized on the fly,
- * gate/up fused with SwiGLU, down fused with the weighted combine and the
- * shared expert) when the layer is IQ2X gate/up with Q2K down, d and f are
- * 256 times a power of two with d <= 8192 and f <= 8192, k <= 32 and the
- * down kernel's staging of h fits in shared memory; B > 1, and every other
- * single-token layer, run the grouped path internally (each touched expert
- * read once; E <= 1024, else DS4MOE_EINVAL).  On the GEMV path x_bf16 is read
- * before the wait on the preceding kernel (see ds4moe_decode_gateup), so x
- * must not be written by the kernel launched just before this call on the
- * same stream; ds4moe_route between the two satisfies this.  Passage: the
- * expert FFN with quantized routed experts and an unquantized shared expert
- * (ds4 news summary, "model weights"; upppp.jp, "asymmetric 2-bit
- * quantization"); single-token generation speed is the pages' headline
+ * routing (ids, weights) from ds4moe_route.
+ *  - GEMV path, for 1 <= B <= 16 when the layer is IQ2X gate/up with Q2K
+ *    down, d and f are 256 times a power of two with d <= 8192 and f <= 8192,
+ *    k <= 32, and the down kernel's staging of h fits in shared memory: per
+ *    token, each selected expert's packed rows are streamed once and
+ *    dequantized on the fly, gate/up fused with SwiGLU, down fused with the
+ *    weighted combine and the shared expert.  Tokens run one after another,
+ *    each with its own h region of the workspace; for such small batches this
+ *    beats the grouped tensor-core path, whose tiles would hold one or two
+ *    tokens each.  x_bf16 is read before the wait on the preceding kernel (see
+ *    ds4moe_decode_gateup), so x must not be written by the kernel launched
+ *    just before this call on the same stream; ds4moe_route between the two
+ *    satisfies this.
+ *  - Grouped path, for B > 16 and for every layer the GEMV path does not
+ *    take: the permuted grouped GEMMs of ds4moe_expert_ffn_grouped (each
+ *    touched expert read once), then the combine; E <= 1024, else
+ *    DS4MOE_EINVAL.
+ * Passage: the expert FFN with quantized routed experts and an unquantized
+ * shared expert (ds4 news summary, "model weights"; upppp.jp, "asymmetric
+ * 2-bit quantization"); single-token generation speed is the pages' headline
  * figure (ds4 news summary, "speed benchmarks"). */
 ds4moe_status ds4moe_expert_ffn_decode(const ds4moe_experts *ex, const void *x_bf16, int B, const int32_t *ids,
                                        const float *weights, int k, float *out, void *ws, size_t ws_bytes,

@@ -107,17 +107,18 @@ def test_decode_gemv_limits_checked_on_host():
 
 def test_grouped_path_expert_limit():
     """The grouped path's offset scan is one CTA of 1024 threads: more than 1024 experts are refused before any
-    launch (and the workspace query returns 0), while the single-token GEMV path, which has no such scan, still
-    takes such a layer."""
+    launch (and the workspace query returns 0) for the batches that need that path, while the GEMV path (batches
+    of up to 16 tokens), which has no such scan, still takes such a layer."""
     lib = ds4moe.lib()
     fake = ctypes.c_void_p(1 << 20)
     big = ds4moe.Experts(256, 512, 2048, 0, 0, 0, 1, 1 << 20, 1 << 21, 1 << 22, 1 << 16, 1 << 16, 1 << 16, 1 << 23,
                          None, None, None)
-    assert lib.ds4moe_workspace_size(ctypes.byref(big), 4, 2) == 0
-    assert lib.ds4moe_workspace_size(ctypes.byref(big), 1, 2) > 0  # B = 1: GEMV path
+    assert lib.ds4moe_workspace_size(ctypes.byref(big), 17, 2) == 0  # B > 16: grouped path only
+    assert lib.ds4moe_workspace_size(ctypes.byref(big), 1, 2) > 0  # B <= 16: GEMV path
+    assert lib.ds4moe_workspace_size(ctypes.byref(big), 16, 2) > 0
     assert lib.ds4moe_expert_ffn_grouped(ctypes.byref(big), fake, 4, fake, fake, 2, fake, fake, None, fake,
                                          1 << 30, None) == 1
-    assert lib.ds4moe_expert_ffn_decode(ctypes.byref(big), fake, 4, fake, fake, 2, fake, fake, 1 << 30, None) == 1
+    assert lib.ds4moe_expert_ffn_decode(ctypes.byref(big), fake, 17, fake, fake, 2, fake, fake, 1 << 30, None) == 1
     q4big = ds4moe.Experts(256, 512, 2048, 0, 2, 2, 2, 1 << 20, 1 << 21, 1 << 22, 1 << 17, 1 << 17, 1 << 17, None,
                            None, None, None)
     assert lib.ds4moe_workspace_size(ctypes.byref(q4big), 1, 2) == 0  # Q4K B = 1 runs the grouped path

@@ -175,8 +175,9 @@ def test_decode_full_size(ds4, decode_layer):
     run_and_compare(ds4, L, x, "decode")
 
 
-@pytest.mark.parametrize("B", [4, 16, 64])
+@pytest.mark.parametrize("B", [2, 3, 4, 16, 17, 64])
 def test_batched_decode(ds4, B):
+    """B <= 16 runs the single-token GEMV pair token by token, larger batches the grouped path (17 and 64)."""
     wl = synth.WORKLOADS["batched"]
     L = synth.make_layer(wl)
     x = synth.activations(wl, B)
