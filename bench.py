@@ -532,7 +532,7 @@ def run_workloads(ds4moe, torch, stream, hbm, tf, peak_kind):
         nb = step_bytes(s, s.k, 1)
         decode = {"B": 1, "tokens_per_s": 1e3 / ms1, "ms_per_token": ms1, "bytes_per_token": nb,
                   "GBps": nb / (ms1 / 1e3) / 1e9, "frac_of_hbm": nb / (ms1 / 1e3) / 1e9 / hbm,
-                  "path": "grouped (no Q4K GEMV yet)", "timing": "mean of %d tokens, L2 flushed between" % n}
+                  "path": "single-token GEMV (Q4K)", "timing": "mean of %d tokens, L2 flushed between" % n}
         return {"workload": "q4: decode layer with Q4K gate/up/down, router bias N(0,1)", "prefill": prefill,
                 "decode": decode, "peak_kind": peak_kind}
 

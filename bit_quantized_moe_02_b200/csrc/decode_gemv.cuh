@@ -36,6 +36,9 @@
 // section; the kernel design is this library's own.
 #pragma once
 #include "common.cuh"
+#include "grouped_common.cuh"  // q4k_field
+
+#include <type_traits>
 
 namespace ds4 {
 
@@ -58,6 +61,11 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
 __device__ __forceinline__ uint2 lds64(uint32_t addr) {
     uint2 v;
     asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+    return v;
+}
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
     return v;
 }
 __device__ __forceinline__ uint2 ldg_nc_v2(const void *p) {
@@ -122,8 +130,9 @@ __host__ __device__ __forceinline__ bool dg_supported_d(int d) {
     const int nblk = d / QK;
     return d % QK == 0 && nblk >= 1 && nblk <= 32 && (nblk & (nblk - 1)) == 0;
 }
-// dynamic shared memory: everything up to the table's end, then x as fp16 (2d bytes) and fp32 (4d bytes)
-__host__ __device__ __forceinline__ int dg_smem_bytes(int d) { return int(DG_TABLE_ABS) + 65536 + d * 6; }
+// dynamic shared memory: everything up to the table's end, then x as fp16 (2d bytes) and fp32 (4d bytes) and the
+// sums of every 8 fp16 activations (d / 2 bytes, Q4K rows only)
+__host__ __device__ __forceinline__ int dg_smem_bytes(int d) { return int(DG_TABLE_ABS) + 65536 + d * 6 + d / 2; }
 
 template <int VPP>
 struct IqRp {  // a lane's slice of one IQ2X row in one pass: VPP 8-vectors
@@ -184,6 +193,80 @@ __device__ __forceinline__ float iq_rp_dot(const IqRp<VPP> &R, const uint4 (&xr)
     return acc;
 }
 
+
+// Q4K rows (gate/up Q4K-style layout): a lane's slice of one row in one pass is 8 VPP weights (VPP words of 8
+// 4-bit codes), inside one 256-weight block, with that block's 12 scale bytes and its d | dmin << 16.
+template <int VPP>
+struct Q4Rp {
+    uint32_t qs[VPP];
+    uint32_t sc[3];
+    uint32_t dm;
+};
+
+// v0: first 8-vector of the slice within the row (a multiple of VPP)
+template <int VPP>
+__device__ __forceinline__ void q4_rp_load(Q4Rp<VPP> &R, const uint8_t *W, const Planes &P, size_t row, int nblk,
+                                           int v0) {
+    const size_t blk = row * size_t(nblk) + v0 / 32;
+    const uint8_t *qp = W + P.off[0] + blk * 128 + (v0 % 32) * 4;
+    if constexpr (VPP == 8) {
+        const uint4 a = ldg_nc_v4(qp), b = ldg_nc_v4(qp + 16);
+        R.qs[0] = a.x; R.qs[1] = a.y; R.qs[2] = a.z; R.qs[3] = a.w;
+        R.qs[4] = b.x; R.qs[5] = b.y; R.qs[6] = b.z; R.qs[7] = b.w;
+    } else if constexpr (VPP == 4) {
+        const uint4 a = ldg_nc_v4(qp);
+        R.qs[0] = a.x; R.qs[1] = a.y; R.qs[2] = a.z; R.qs[3] = a.w;
+    } else if constexpr (VPP == 2) {
+        const uint2 a = ldg_nc_v2(qp);
+        R.qs[0] = a.x; R.qs[1] = a.y;
+    } else {
+        R.qs[0] = ldg_nc_u32(qp);
+    }
+    const uint8_t *sp = W + P.off[1] + blk * 12;
+    R.sc[0] = ldg_nc_u32(sp);
+    R.sc[1] = ldg_nc_u32(sp + 4);
+    R.sc[2] = ldg_nc_u32(sp + 8);
+    R.dm = ldg_nc_u32(W + P.off[2] + blk * 4);
+}
+
+// Dot product of a lane's Q4K row slice with its activations xr (fp16 pairs, natural order) and their sums over
+// 8-weight pieces xs8: w = d * sc * q - dmin * m per 32-weight sub-block, so the slice contributes
+// d * sum_sb sc * (q . x) - dmin * sum_sb m * (sum x).  q comes from a byte -> (low nibble, high nibble) fp16-pair
+// table (one 4-byte lane slot per lane: conflict-free); q . x in fp16 inside a sub-block (each half adds at most
+// 16 products of q <= 15 and |x| < 64), the rest in fp32.
+template <int VPP>
+__device__ __forceinline__ float q4_rp_dot(const Q4Rp<VPP> &R, const uint4 (&xr)[VPP], const float (&xs8)[VPP], int v0,
+                                           uint32_t lane_tbl) {
+    constexpr int NSB = VPP >= 4 ? VPP / 4 : 1, VS = VPP >= 4 ? 4 : VPP;
+    const int sb0 = (v0 % 32) / 4;  // first sub-block of the slice inside its block
+    float A = 0.f, B = 0.f;
+#pragma unroll
+    for (int i = 0; i < NSB; i++) {
+        __half2 a = __float2half2_rn(0.f), b = a;
+        float xsum = 0.f;
+#pragma unroll
+        for (int j = 0; j < VS; j++) {
+            const int v = i * 4 + j;
+            const uint32_t t0 = lds32(__byte_perm(R.qs[v], lane_tbl, 0x7604));
+            const uint32_t t1 = lds32(__byte_perm(R.qs[v], lane_tbl, 0x7614));
+            const uint32_t t2 = lds32(__byte_perm(R.qs[v], lane_tbl, 0x7624));
+            const uint32_t t3 = lds32(__byte_perm(R.qs[v], lane_tbl, 0x7634));
+            a = __hfma2(u32_as_half2(t0), u32_as_half2(xr[v].x), a);
+            b = __hfma2(u32_as_half2(t1), u32_as_half2(xr[v].y), b);
+            a = __hfma2(u32_as_half2(t2), u32_as_half2(xr[v].z), a);
+            b = __hfma2(u32_as_half2(t3), u32_as_half2(xr[v].w), b);
+            xsum += xs8[v];
+        }
+        const int sb = sb0 + i;
+        const float sc = float(q4k_field(R.sc[0], R.sc[1], R.sc[2], 6 * sb));
+        const float mn = float(q4k_field(R.sc[0], R.sc[1], R.sc[2], 48 + 6 * sb));
+        const float2 s2 = __half22float2(__hadd2(a, b));
+        A = fmaf(sc, s2.x + s2.y, A);
+        B = fmaf(mn, xsum, B);
+    }
+    return half_bits_to_float(uint16_t(R.dm & 0xFFFF)) * A - half_bits_to_float(uint16_t(R.dm >> 16)) * B;
+}
+
 __device__ __forceinline__ float bf16x8_dot(const uint4 w, const float4 a, const float4 b) {
     float s = bf16_lo(w.x) * a.x;
     s = fmaf(bf16_hi(w.x), a.y, s);
@@ -198,7 +281,7 @@ __device__ __forceinline__ float bf16x8_dot(const uint4 w, const float4 a, const
 
 // Units of NR row pairs: shared-expert units first (rows NR u .. NR u + NR - 1 of Gs, Us), then routed units
 // (expert slot j, rows NR i ..).  Row-matrix index rr = 2 * (row - first row) + (0 gate, 1 up).
-template <int VPP, int NR>
+template <int FMT, int VPP, int NR>
 __global__ void __launch_bounds__(DG_THREADS, 1)
     decode_gateup_kernel(const ExpertsDev ex, const __nv_bfloat16 *__restrict__ x, const int32_t *ids, int k,
                          float *__restrict__ h_out, float *__restrict__ hs_out) {
@@ -212,7 +295,9 @@ __global__ void __launch_bounds__(DG_THREADS, 1)
     uint8_t *tbl = smem + (DG_TABLE_ABS - sbase);
     __half *x16 = reinterpret_cast<__half *>(tbl + 65536);
     float *x32 = reinterpret_cast<float *>(tbl + 65536 + d * 2);
+    float *xs8 = reinterpret_cast<float *>(tbl + 65536 + d * 6);  // Q4K: sums of every 8 fp16 activations
     const uint32_t x16_s = DG_TABLE_ABS + 65536;
+    constexpr bool Q4 = FMT == DS4MOE_FMT_Q4K;
 
     constexpr int NRR = 2 * NR;      // row-matrices per unit
     constexpr int LPV = 32 / NRR;    // lanes that hold one row-matrix sum after the reduce-scatter
@@ -231,7 +316,7 @@ __global__ void __launch_bounds__(DG_THREADS, 1)
     // that puts max |x| in [32, 64)
     static_assert(DG_THREADS >= 512, "two threads per codebook entry");
     const int e_cb = tid >> 1;  // threads 0 .. 511 build the table
-    const uint2 raw = tid < 512 ? *reinterpret_cast<const uint2 *>(ex.codebook + e_cb * 8) : make_uint2(0, 0);
+    const uint2 raw = !Q4 && tid < 512 ? *reinterpret_cast<const uint2 *>(ex.codebook + e_cb * 8) : make_uint2(0, 0);
     constexpr int XPT = (DG_MAX_D + DG_THREADS * 8 - 1) / (DG_THREADS * 8);  // 8-element chunks per thread
     uint4 xv[XPT];
 #pragma unroll
@@ -239,7 +324,14 @@ __global__ void __launch_bounds__(DG_THREADS, 1)
         const int i = (tid + c * DG_THREADS) * 8;
         if (i < d) xv[c] = *reinterpret_cast<const uint4 *>(x + i);
     }
-    if (tid < 512) {
+    if constexpr (Q4) {
+        // byte -> (low nibble, high nibble) as an fp16 pair: entry b, lane slot s at DG_TABLE_ABS + b * 256 + s * 4
+        for (int i = tid; i < 256 * 32; i += DG_THREADS) {
+            const int b = i >> 5;
+            *reinterpret_cast<uint32_t *>(tbl + b * 256 + (i & 31) * 4) =
+                half2_as_u32(__floats2half2_rn(float(b & 15), float(b >> 4)));
+        }
+    } else if (tid < 512) {
         const uint32_t b[2] = {raw.x, raw.y};
         __half2 hv[4];
 #pragma unroll
@@ -278,18 +370,24 @@ __global__ void __launch_bounds__(DG_THREADS, 1)
         const int i = (tid + c * DG_THREADS) * 8;
         if (i < d) {
             const uint4 v = xv[c];
+            const __half2 h0 = __floats2half2_rn(bf16_lo(v.x) * xs, bf16_hi(v.x) * xs);
+            const __half2 h1 = __floats2half2_rn(bf16_lo(v.y) * xs, bf16_hi(v.y) * xs);
+            const __half2 h2 = __floats2half2_rn(bf16_lo(v.z) * xs, bf16_hi(v.z) * xs);
+            const __half2 h3 = __floats2half2_rn(bf16_lo(v.w) * xs, bf16_hi(v.w) * xs);
             reinterpret_cast<uint4 *>(x16)[swz16(i / 8)] =
-                make_uint4(half2_as_u32(__floats2half2_rn(bf16_lo(v.x) * xs, bf16_hi(v.x) * xs)),
-                           half2_as_u32(__floats2half2_rn(bf16_lo(v.y) * xs, bf16_hi(v.y) * xs)),
-                           half2_as_u32(__floats2half2_rn(bf16_lo(v.z) * xs, bf16_hi(v.z) * xs)),
-                           half2_as_u32(__floats2half2_rn(bf16_lo(v.w) * xs, bf16_hi(v.w) * xs)));
+                make_uint4(half2_as_u32(h0), half2_as_u32(h1), half2_as_u32(h2), half2_as_u32(h3));
+            if constexpr (Q4) {
+                const float2 f0 = __half22float2(h0), f1 = __half22float2(h1), f2 = __half22float2(h2),
+                             f3 = __half22float2(h3);
+                xs8[i / 8] = ((f0.x + f0.y) + (f1.x + f1.y)) + ((f2.x + f2.y) + (f3.x + f3.y));
+            }
         }
     }
     __syncthreads();
 
     // the down kernel may launch as CTAs of this grid finish (it waits for the whole grid before reading h)
     pdl_launch_dependents();
-    const uint32_t lane_tbl = DG_TABLE_ABS | uint32_t((lane & 15) * 16);
+    const uint32_t lane_tbl = DG_TABLE_ABS | uint32_t(Q4 ? lane * 4 : (lane & 15) * 16);
     bool waited = false;
     for (int u = u_first; u < n_all; u += nW) {
         float acc[NRR];
@@ -335,21 +433,31 @@ __global__ void __launch_bounds__(DG_THREADS, 1)
         }
         const uint8_t *G = ex.gate + size_t(e) * ex.gate_stride, *U = ex.up + size_t(e) * ex.up_stride;
         const int T = npass * NRR;
-        auto load = [&](IqRp<VPP> &R, int t) {
+        using Rp = typename std::conditional<Q4, Q4Rp<VPP>, IqRp<VPP>>::type;
+        auto load = [&](Rp &R, int t) {
             const int rr = t % NRR;
-            iq_rp_load<VPP>(R, rr & 1 ? U : G, ex.pg, r0 + (rr >> 1), nblk, (t / NRR) * 32 * VPP + lane * VPP);
+            if constexpr (Q4)
+                q4_rp_load<VPP>(R, rr & 1 ? U : G, ex.pg, r0 + (rr >> 1), nblk, (t / NRR) * 32 * VPP + lane * VPP);
+            else
+                iq_rp_load<VPP>(R, rr & 1 ? U : G, ex.pg, r0 + (rr >> 1), nblk, (t / NRR) * 32 * VPP + lane * VPP);
         };
-        IqRp<VPP> ring[DG_RING];
+        Rp ring[DG_RING];
 #pragma unroll
         for (int s = 0; s < DG_RING; s++) load(ring[s], s);
         for (int p = 0; p < npass; p++) {
             const int v0 = p * 32 * VPP + lane * VPP;
             uint4 xr[VPP];
+            float xsv[VPP];
 #pragma unroll
             for (int v = 0; v < VPP; v++) xr[v] = lds128(x16_s + swz16(v0 + v) * 16);
+            if constexpr (Q4) {
+#pragma unroll
+                for (int v = 0; v < VPP; v++) xsv[v] = xs8[v0 + v];
+            }
 #pragma unroll
             for (int rr = 0; rr < NRR; rr++) {
-                acc[rr] += iq_rp_dot<VPP>(ring[rr % DG_RING], xr, v0, lane_tbl);
+                if constexpr (Q4) acc[rr] += q4_rp_dot<VPP>(ring[rr % DG_RING], xr, xsv, v0, lane_tbl);
+                else acc[rr] += iq_rp_dot<VPP>(ring[rr % DG_RING], xr, v0, lane_tbl);
                 const int tn = p * NRR + rr + DG_RING;
                 if (tn < T) load(ring[rr % DG_RING], tn);
             }
@@ -462,6 +570,77 @@ __device__ __forceinline__ float qk_rp_dot(const QkRp<EPL> &R, const uint32_t (&
     return dd * A - dmin * B;
 }
 
+
+// Q4K down rows: a lane's slice of one row in one pass is EPL weights (EPL / 8 words of 4-bit codes) inside one
+// 256-weight block, with that block's 12 scale bytes and d | dmin << 16.
+template <int EPL>
+struct Q4DRp {
+    static constexpr int NQ = EPL / 8;
+    uint32_t qs[NQ];
+    uint32_t sc[3];
+    uint32_t dm;
+};
+
+template <int EPL>
+__device__ __forceinline__ void q4d_rp_load(Q4DRp<EPL> &R, const uint8_t *W, const Planes &P, size_t row, int nblkf,
+                                            int e0) {
+    const size_t blk = row * size_t(nblkf) + e0 / 256;
+    const uint8_t *qp = W + P.off[0] + blk * 128 + (e0 % 256) / 2;
+    if constexpr (EPL == 64) {
+        const uint4 a = ldg_nc_v4(qp), b = ldg_nc_v4(qp + 16);
+        R.qs[0] = a.x; R.qs[1] = a.y; R.qs[2] = a.z; R.qs[3] = a.w;
+        R.qs[4] = b.x; R.qs[5] = b.y; R.qs[6] = b.z; R.qs[7] = b.w;
+    } else if constexpr (EPL == 32) {
+        const uint4 a = ldg_nc_v4(qp);
+        R.qs[0] = a.x; R.qs[1] = a.y; R.qs[2] = a.z; R.qs[3] = a.w;
+    } else if constexpr (EPL == 16) {
+        const uint2 a = ldg_nc_v2(qp);
+        R.qs[0] = a.x; R.qs[1] = a.y;
+    } else {
+        R.qs[0] = ldg_nc_u32(qp);
+    }
+    const uint8_t *sp = W + P.off[1] + blk * 12;
+    R.sc[0] = ldg_nc_u32(sp);
+    R.sc[1] = ldg_nc_u32(sp + 4);
+    R.sc[2] = ldg_nc_u32(sp + 8);
+    R.dm = ldg_nc_u32(W + P.off[2] + blk * 4);
+}
+
+// sum over the slice of w_i * hh_i with w = d * sc * q - dmin * m per 32-weight sub-block (hh: the lane's staged
+// h, fp16 pairs in natural order; hs8: sums of every 8 staged values); q from the byte -> fp16-pair table
+template <int EPL>
+__device__ __forceinline__ float q4d_rp_dot(const Q4DRp<EPL> &R, const uint32_t (&hh)[EPL / 2],
+                                            const float (&hs8)[EPL / 8], int e0, uint32_t lane_tbl) {
+    constexpr int NSB = EPL >= 32 ? EPL / 32 : 1, WS = EPL >= 32 ? 4 : EPL / 8;  // sub-blocks, words per sub-block
+    const int sb0 = (e0 % 256) / 32;
+    float A = 0.f, B = 0.f;
+#pragma unroll
+    for (int i = 0; i < NSB; i++) {
+        __half2 a = __float2half2_rn(0.f), b = a;
+        float hsum = 0.f;
+#pragma unroll
+        for (int j = 0; j < WS; j++) {
+            const int w = i * 4 + j;  // word: weights 8 w .. 8 w + 7
+            const uint32_t t0 = lds32(__byte_perm(R.qs[w], lane_tbl, 0x7604));
+            const uint32_t t1 = lds32(__byte_perm(R.qs[w], lane_tbl, 0x7614));
+            const uint32_t t2 = lds32(__byte_perm(R.qs[w], lane_tbl, 0x7624));
+            const uint32_t t3 = lds32(__byte_perm(R.qs[w], lane_tbl, 0x7634));
+            a = __hfma2(u32_as_half2(t0), u32_as_half2(hh[4 * w]), a);
+            b = __hfma2(u32_as_half2(t1), u32_as_half2(hh[4 * w + 1]), b);
+            a = __hfma2(u32_as_half2(t2), u32_as_half2(hh[4 * w + 2]), a);
+            b = __hfma2(u32_as_half2(t3), u32_as_half2(hh[4 * w + 3]), b);
+            hsum += hs8[w];
+        }
+        const int sb = sb0 + i;
+        const float sc = float(q4k_field(R.sc[0], R.sc[1], R.sc[2], 6 * sb));
+        const float mn = float(q4k_field(R.sc[0], R.sc[1], R.sc[2], 48 + 6 * sb));
+        const float2 s2 = __half22float2(__hadd2(a, b));
+        A = fmaf(sc, s2.x + s2.y, A);
+        B = fmaf(mn, hsum, B);
+    }
+    return half_bits_to_float(uint16_t(R.dm & 0xFFFF)) * A - half_bits_to_float(uint16_t(R.dm >> 16)) * B;
+}
+
 // the lane's staged slice (EPL fp16 and EPL / 8 sums) at shared addresses hq_addr, hs_addr
 template <int EPL>
 __device__ __forceinline__ void dd_slice_load(uint32_t hq_addr, uint32_t hs_addr, uint32_t (&hh)[EPL / 2],
@@ -488,11 +667,12 @@ __device__ __forceinline__ void dd_slice_load(uint32_t hq_addr, uint32_t hs_addr
     }
 }
 
-template <int EPL>
+template <int FMT, int EPL>
 __global__ void __launch_bounds__(DD_THREADS, 1)
     decode_down_kernel(const ExpertsDev ex, const float *h, const float *hs_in, const int32_t *ids, const float *wts,
                        int k, float *__restrict__ out) {
     extern __shared__ __align__(1024) uint8_t smem[];
+    constexpr bool Q4 = FMT == DS4MOE_FMT_Q4K;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int d = ex.d, f = ex.f, fs = ex.fs;
     const int nblkf = f / QK;
@@ -510,12 +690,18 @@ __global__ void __launch_bounds__(DD_THREADS, 1)
     if (fs > 0 && u_first < n_units && lane == 0)
         prefetch_l2(ex.sh_down + size_t(u_first) * DD_ROWS * fs, uint32_t(DD_ROWS * fs * 2));
 
-    // byte -> 4 fp16 table: entry b holds q_i = (b >> 2i) & 3, lane slot s at DD_TABLE_ABS + b * 256 + s * 8
+    // Q2K: byte -> 4 fp16 table, entry b holds q_i = (b >> 2i) & 3, lane slot s at DD_TABLE_ABS + b * 256 + s * 8;
+    // Q4K: byte -> (low nibble, high nibble) as an fp16 pair, lane slot s at DD_TABLE_ABS + b * 256 + s * 4
     for (int i = tid; i < 256 * 32; i += DD_THREADS) {
         const int b = i >> 5;
-        const __half2 lo = __floats2half2_rn(float(b & 3), float((b >> 2) & 3));
-        const __half2 hi = __floats2half2_rn(float((b >> 4) & 3), float((b >> 6) & 3));
-        *reinterpret_cast<uint2 *>(tb + b * 256 + (i & 31) * 8) = make_uint2(half2_as_u32(lo), half2_as_u32(hi));
+        if constexpr (Q4) {
+            *reinterpret_cast<uint32_t *>(tb + b * 256 + (i & 31) * 4) =
+                half2_as_u32(__floats2half2_rn(float(b & 15), float(b >> 4)));
+        } else {
+            const __half2 lo = __floats2half2_rn(float(b & 3), float((b >> 2) & 3));
+            const __half2 hi = __floats2half2_rn(float((b >> 4) & 3), float((b >> 6) & 3));
+            *reinterpret_cast<uint2 *>(tb + b * 256 + (i & 31) * 8) = make_uint2(half2_as_u32(lo), half2_as_u32(hi));
+        }
     }
 
     pdl_wait();  // h and hs come from the gate/up kernel, ids and weights from the router
@@ -525,12 +711,17 @@ __global__ void __launch_bounds__(DD_THREADS, 1)
     // Rings of the unit in progress: routed steps n and n + 1 (both rows), shared passes p .. p + 3 (both rows).
     // (Filling the first unit's rings before the staging below was measured slower: those loads then compete
     // with the staging's reads of h, which every warp waits for.)
-    QkRp<EPL> rg[2][2];
+    using Rp = typename std::conditional<Q4, Q4DRp<EPL>, QkRp<EPL>>::type;
+    Rp rg[2][2];
     uint4 sr[4][2];
     int pn = 0, jn = 0;  // next routed step to load
-    auto rload = [&](QkRp<EPL> &R, int e, size_t row, int p) {
-        if (e >= 0 && e < ex.E)
-            qk_rp_load<EPL>(R, ex.down + size_t(e) * ex.down_stride, ex.pd, row, nblkf, p * 32 * EPL + lane * EPL);
+    auto rload = [&](Rp &R, int e, size_t row, int p) {
+        if (e >= 0 && e < ex.E) {
+            if constexpr (Q4)
+                q4d_rp_load<EPL>(R, ex.down + size_t(e) * ex.down_stride, ex.pd, row, nblkf, p * 32 * EPL + lane * EPL);
+            else
+                qk_rp_load<EPL>(R, ex.down + size_t(e) * ex.down_stride, ex.pd, row, nblkf, p * 32 * EPL + lane * EPL);
+        }
     };
     auto prime = [&](int u, const int *idv) {
         const size_t r0 = size_t(u) * DD_ROWS;
@@ -604,7 +795,7 @@ __global__ void __launch_bounds__(DD_THREADS, 1)
         reinterpret_cast<float4 *>(hsl)[swz16(i / 4)] = *reinterpret_cast<const float4 *>(hs_in + i);
     __syncthreads();
 
-    const uint32_t lane_tbl = DD_TABLE_ABS | uint32_t(lane * 8);
+    const uint32_t lane_tbl = DD_TABLE_ABS | uint32_t(lane * (Q4 ? 4 : 8));
     const uint32_t hq_lane = DD_TABLE_ABS + uint32_t(L.hq + lane * L.hq_sb);
     const uint32_t hs_lane = DD_TABLE_ABS + uint32_t(L.hsum + lane * L.hs_sb);
     for (int u = u_first; u < n_units; u += nW) {
@@ -647,8 +838,14 @@ __global__ void __launch_bounds__(DD_THREADS, 1)
                     const int e = eid[j];
                     if (e >= 0 && e < ex.E) {
                         const float w = wsc[j];
-                        acc0 = fmaf(w, qk_rp_dot<EPL>(rg[s][0], hh, hs8, lane_tbl), acc0);
-                        acc1 = fmaf(w, qk_rp_dot<EPL>(rg[s][1], hh, hs8, lane_tbl), acc1);
+                        if constexpr (Q4) {
+                            const int e0 = p * 32 * EPL + lane * EPL;
+                            acc0 = fmaf(w, q4d_rp_dot<EPL>(rg[s][0], hh, hs8, e0, lane_tbl), acc0);
+                            acc1 = fmaf(w, q4d_rp_dot<EPL>(rg[s][1], hh, hs8, e0, lane_tbl), acc1);
+                        } else {
+                            acc0 = fmaf(w, qk_rp_dot<EPL>(rg[s][0], hh, hs8, lane_tbl), acc0);
+                            acc1 = fmaf(w, qk_rp_dot<EPL>(rg[s][1], hh, hs8, lane_tbl), acc1);
+                        }
                     }
                     if (n0 + s + 2 < NS) {
                         const int en = eid[jn];

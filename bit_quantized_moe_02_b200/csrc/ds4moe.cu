@@ -184,7 +184,9 @@ ExpertsDev to_dev(const ds4moe_experts *ex) {
 // The single-token GEMV kernels cover IQ2X gate/up with Q2K down, d <= 8192, and a down-kernel staging area
 // that fits in shared memory; everything else runs the grouped path with one token.
 bool decode_gemv_supported(const ds4moe_experts *ex, int k) {
-    if (ex->fmt_gate != DS4MOE_FMT_IQ2X || ex->fmt_down != DS4MOE_FMT_Q2K || k > 32) return false;
+    const bool iq = ex->fmt_gate == DS4MOE_FMT_IQ2X && ex->fmt_down == DS4MOE_FMT_Q2K;
+    const bool q4 = ex->fmt_gate == DS4MOE_FMT_Q4K && ex->fmt_down == DS4MOE_FMT_Q4K;
+    if (!(iq || q4) || k > 32) return false;
     if (!dg_supported_d(ex->d) || !dd_supported_f(ex->f)) return false;
     return dd_layout(k, ex->f, ex->f_shared).total <= 200 * 1024;
 }
@@ -610,8 +612,14 @@ ds4moe_status ds4moe_decode_gateup(const ds4moe_experts *ex, const void *x_bf16,
     const __nv_bfloat16 *x = static_cast<const __nv_bfloat16 *>(x_bf16);
     const int smem = dg_smem_bytes(ex->d);
     const int vpp = ex->d / QK < 8 ? ex->d / QK : 8;  // 8-vectors of a row per lane and pass
-    auto kern = vpp == 8 ? decode_gateup_kernel<8, DG_ROWS> : vpp == 4 ? decode_gateup_kernel<4, DG_ROWS>
-              : vpp == 2 ? decode_gateup_kernel<2, DG_ROWS> : decode_gateup_kernel<1, DG_ROWS>;
+    using GK = void (*)(const ExpertsDev, const __nv_bfloat16 *, const int32_t *, int, float *, float *);
+    GK kern;
+    if (ex->fmt_gate == DS4MOE_FMT_Q4K)
+        kern = vpp == 8 ? decode_gateup_kernel<DS4MOE_FMT_Q4K, 8, DG_ROWS> : vpp == 4 ? decode_gateup_kernel<DS4MOE_FMT_Q4K, 4, DG_ROWS>
+             : vpp == 2 ? decode_gateup_kernel<DS4MOE_FMT_Q4K, 2, DG_ROWS> : decode_gateup_kernel<DS4MOE_FMT_Q4K, 1, DG_ROWS>;
+    else
+        kern = vpp == 8 ? decode_gateup_kernel<DS4MOE_FMT_IQ2X, 8, DG_ROWS> : vpp == 4 ? decode_gateup_kernel<DS4MOE_FMT_IQ2X, 4, DG_ROWS>
+             : vpp == 2 ? decode_gateup_kernel<DS4MOE_FMT_IQ2X, 2, DG_ROWS> : decode_gateup_kernel<DS4MOE_FMT_IQ2X, 1, DG_ROWS>;
     if (!set_smem(kern, smem)) return DS4MOE_ECUDA;
     const cudaError_t err =
         launch_pdl(kern, dim3(num_sms()), dim3(DG_THREADS), size_t(smem), cs(stream), D, x, ids, k, h, hs);
@@ -638,8 +646,14 @@ ds4moe_status ds4moe_decode_down(const ds4moe_experts *ex, const int32_t *ids, c
     const float *hs = reinterpret_cast<const float *>(w8 + W.hs);
     const int smem = dd_layout(k, ex->f, ex->f_shared).total;
     const int epl = dd_epl(ex->f);  // weights of a row per lane and pass
-    auto kern = epl == 64 ? decode_down_kernel<64> : epl == 32 ? decode_down_kernel<32>
-              : epl == 16 ? decode_down_kernel<16> : decode_down_kernel<8>;
+    using DK = void (*)(const ExpertsDev, const float *, const float *, const int32_t *, const float *, int, float *);
+    DK kern;
+    if (ex->fmt_down == DS4MOE_FMT_Q4K)
+        kern = epl == 64 ? decode_down_kernel<DS4MOE_FMT_Q4K, 64> : epl == 32 ? decode_down_kernel<DS4MOE_FMT_Q4K, 32>
+             : epl == 16 ? decode_down_kernel<DS4MOE_FMT_Q4K, 16> : decode_down_kernel<DS4MOE_FMT_Q4K, 8>;
+    else
+        kern = epl == 64 ? decode_down_kernel<DS4MOE_FMT_Q2K, 64> : epl == 32 ? decode_down_kernel<DS4MOE_FMT_Q2K, 32>
+             : epl == 16 ? decode_down_kernel<DS4MOE_FMT_Q2K, 16> : decode_down_kernel<DS4MOE_FMT_Q2K, 8>;
     if (!set_smem(kern, smem)) return DS4MOE_ECUDA;
     const cudaError_t err = launch_pdl(kern, dim3(num_sms()), dim3(DD_THREADS), size_t(smem), cs(stream), D, h, hs,
                                        ids, weights, k, out);

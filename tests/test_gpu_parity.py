@@ -155,6 +155,17 @@ def test_decode_gemv_shapes(ds4, d, f, fs, E, k):
     run_and_compare(ds4, L, x, "decode")
 
 
+@pytest.mark.parametrize("d,f,fs,E,k", [(4096, 2048, 2048, 16, 8), (2048, 1024, 512, 16, 4), (1024, 256, 0, 8, 2)])
+def test_q4k_decode_gemv(ds4, d, f, fs, E, k):
+    """Single-token decode of Q4K layers through the GEMV kernels (the decode layer's shape with 16 experts, then
+    smaller lane slices: 32 and 8 weights per lane in the down kernel, 4 and 2 vectors per lane in gate/up)."""
+    shape = synth.LayerShape(d=d, E=E, f=f, k=k, f_shared=fs, fmt_gate="q4k", fmt_up="q4k", fmt_down="q4k")
+    L = layer_of(shape, 1.0, 81 + d)
+    x = synth.f32_to_bf16_bits(synth.rng(8, d).normal(size=(4, d)).astype(np.float32))
+    run_and_compare(ds4, L, x, "decode")
+    run_and_compare(ds4, L, x, "batched")  # B = 4: token by token through the same kernels
+
+
 def test_q4k_layer_small(ds4):
     shape = synth.LayerShape(d=512, E=8, f=768, k=2, f_shared=256, fmt_gate="q4k", fmt_up="q4k", fmt_down="q4k")
     L = layer_of(shape, 1.0, 77)
