@@ -188,7 +188,8 @@ size_t ds4moe_workspace_size(const ds4moe_experts *ex, int T, int k);
 /* Decode: out[B x d] (fp32) = the full layer output for B tokens, given the
  * routing (ids, weights) from ds4moe_route.
  *  - GEMV path, for 1 <= B <= 16 when the layer is IQ2X gate/up with Q2K
- *    down, d and f are 256 times a power of two with d <= 8192 and f <= 8192,
+ *    down, or Q4K throughout, d and f are 256 times a power of two with
+ *    d <= 8192 and f <= 8192,
  *    k <= 32, and the down kernel's staging of h fits in shared memory: per
  *    token, each selected expert's packed rows are streamed once and
  *    dequantized on the fly, gate/up fused with SwiGLU, down fused with the

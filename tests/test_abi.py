@@ -81,8 +81,8 @@ def test_host_side_argument_checks():
 
 def test_decode_gemv_limits_checked_on_host():
     """The single-token GEMV halves refuse layers outside their limits before any launch: d and f 256 times a power
-    of two up to 8192, gate/up IQ2X with Q2K down, k <= 32; the combined decode call then runs the grouped path
-    instead (its own checks)."""
+    of two up to 8192, IQ2X gate/up with Q2K down or Q4K throughout, k <= 32; the combined decode call then runs
+    the grouped path instead (its own checks)."""
     lib = ds4moe.lib()
     fake = ctypes.c_void_p(1 << 20)
 
@@ -94,8 +94,10 @@ def test_decode_gemv_limits_checked_on_host():
         ex = experts(d, f)
         assert lib.ds4moe_decode_gateup(ctypes.byref(ex), fake, fake, 2, fake, 1 << 30, None) == 2, (d, f)
         assert lib.ds4moe_decode_down(ctypes.byref(ex), fake, fake, 2, fake, fake, 1 << 30, None) == 2, (d, f)
-    q4 = experts(512, 512, fmt_gate=2, fmt_down=2)  # Q4K has no GEMV kernel
-    assert lib.ds4moe_decode_gateup(ctypes.byref(q4), fake, fake, 2, fake, 1 << 30, None) == 2
+    mixed = experts(512, 512, fmt_gate=2, fmt_down=1)  # Q4K gate/up with Q2K down: no GEMV kernel pair
+    assert lib.ds4moe_decode_gateup(ctypes.byref(mixed), fake, fake, 2, fake, 1 << 30, None) == 2
+    mixed = experts(512, 512, fmt_gate=0, fmt_down=2)  # IQ2X gate/up with Q4K down
+    assert lib.ds4moe_decode_down(ctypes.byref(mixed), fake, fake, 2, fake, fake, 1 << 30, None) == 2
     ex = experts(512, 512)
     assert lib.ds4moe_decode_gateup(ctypes.byref(ex), fake, fake, 40, fake, 1 << 30, None) == 1  # k > E
     # workspace: h (k*f floats) and the shared expert's h, each rounded to 256 bytes
@@ -119,10 +121,10 @@ def test_grouped_path_expert_limit():
     assert lib.ds4moe_expert_ffn_grouped(ctypes.byref(big), fake, 4, fake, fake, 2, fake, fake, None, fake,
                                          1 << 30, None) == 1
     assert lib.ds4moe_expert_ffn_decode(ctypes.byref(big), fake, 17, fake, fake, 2, fake, fake, 1 << 30, None) == 1
-    q4big = ds4moe.Experts(256, 512, 2048, 0, 2, 2, 2, 1 << 20, 1 << 21, 1 << 22, 1 << 17, 1 << 17, 1 << 17, None,
-                           None, None, None)
-    assert lib.ds4moe_workspace_size(ctypes.byref(q4big), 1, 2) == 0  # Q4K B = 1 runs the grouped path
-    assert lib.ds4moe_expert_ffn_decode(ctypes.byref(q4big), fake, 1, fake, fake, 2, fake, fake, 1 << 30,
+    mixed = ds4moe.Experts(256, 512, 2048, 0, 2, 2, 1, 1 << 20, 1 << 21, 1 << 22, 1 << 17, 1 << 17, 1 << 17, None,
+                           None, None, None)  # Q4K gate/up with Q2K down: even B = 1 needs the grouped path
+    assert lib.ds4moe_workspace_size(ctypes.byref(mixed), 1, 2) == 0
+    assert lib.ds4moe_expert_ffn_decode(ctypes.byref(mixed), fake, 1, fake, fake, 2, fake, fake, 1 << 30,
                                         None) == 1
 
 
