@@ -187,6 +187,21 @@ def oracle_tokens_per_s(wl, n_tokens, nthreads, seed_stream=7):
     return n_tokens / dt, dt
 
 
+def workload_cpu_baselines(cores):
+    """The oracle timed on each other workload's layer (bounded samples of a few seconds each, all host threads):
+    tokens/s on the tiny layer, on the batched-decode layer (router bias N(0,1); the oracle's per-token cost does
+    not depend on the batch size), on the prefill layer (tokens of the T=4096 input) and on the Q4K layer."""
+    res = {}
+    for name, per_thread in (("tiny", 256), ("batched", 4), ("prefill", 4), ("q4", 2)):
+        wl = synth.WORKLOADS[name]
+        n = per_thread * cores
+        tps, dt = oracle_tokens_per_s(wl, n, cores)
+        res[name] = {"value": tps, "unit": UNIT, "cores": cores, "kind": "oracle",
+                     "sample": "%d tokens of the %s workload's layer 0 (%d per host thread), %.1f s"
+                               % (n, name, per_thread, dt)}
+    return res
+
+
 def run_reference(args, ws, rank):
     wl = synth.WORKLOADS["decode"]
     if rank != 0:
@@ -358,6 +373,11 @@ def run_ours(args, ws, rank, local):
         tps, dt = oracle_tokens_per_s(wl, n_cpu, cores)
         cpu = {"value": tps, "unit": UNIT, "cores": cores, "kind": "oracle",
                "sample": "%d decode tokens of layer 0 (12 per host thread), %.1f s" % (n_cpu, dt)}
+        if isinstance(workloads, dict) and "error" not in workloads:
+            for name, cb in workload_cpu_baselines(cores).items():
+                entry = workloads.get(name) if name != "prefill" else prefill
+                if isinstance(entry, dict) and "error" not in entry:
+                    entry["cpu_baseline"] = cb
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": t_max / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -393,27 +413,45 @@ def run_prefill(args, ds4moe, torch, stream, tf, tf_sus, peak_kind):
     inv = torch.empty(T * s.k, dtype=torch.int32, device="cuda")
     ys = torch.empty((T, s.d), dtype=torch.float32, device="cuda")
     out = torch.empty((T, s.d), dtype=torch.float32, device="cuda")
+
+    def deterministic():
+        ids, w = D.route(x, ids=D.ids_buf[:T], weights=D.w_buf[:T])
+        ds4moe.expert_ffn_grouped(D.ex, x, ids, w, D.ws, y_perm, inv, ys)
+        ds4moe.combine(y_perm, inv, ys, T, s.d, s.k, out=out)
+
+    def fused():
+        D.forward_fused(x, out=out)
+
+    flops = 2 * 3 * s.d * s.f * T * s.k + 2 * 3 * s.d * s.f_shared * T + 2 * T * s.E * s.d
+    res = {"workload": "prefill T=%d, same layer, router bias N(0,1)" % T, "peak_tflops": tf, "peak_kind": peak_kind,
+           "flops_per_step": flops}
+    for name, step in (("deterministic", deterministic), ("fused", fused)):
+        ms = device_ms(torch, stream, step, warmup=3, n=10)
+        assert ds4moe.last_device_error() == 0
+        res[name] = {"tokens_per_s": T / (ms / 1e3), "ms_per_step": ms, "tflops": flops / (ms / 1e3) / 1e12,
+                     "frac_of_bf16_peak": flops / (ms / 1e3) / 1e12 / tf}
+    res["deterministic"]["calls"] = "route, expert_ffn_grouped (y_perm, y_shared), combine (fixed summation order)"
+    res["fused"]["calls"] = "route, expert_ffn_grouped_fused (down GEMM adds into out; atomic summation order)"
+    best = min(("deterministic", "fused"), key=lambda n: res[n]["ms_per_step"])
+    res.update({k: res[best][k] for k in ("tokens_per_s", "ms_per_step", "tflops", "frac_of_bf16_peak")})
+    res["headline_mode"] = best
+    del D
+    return res
+
+
+def device_ms(torch, stream, step, warmup, n):
+    """Mean device time of n back-to-back calls of step() on stream (CUDA events), after warmup calls."""
     with torch.cuda.stream(stream):
-        def step():
-            ids, w = D.route(x)
-            ds4moe.expert_ffn_grouped(D.ex, x, ids, w, D.ws, y_perm, inv, ys)
-            ds4moe.combine(y_perm, inv, ys, T, s.d, s.k, out=out)
-        for _ in range(3):
+        for _ in range(warmup):
             step()
         stream.synchronize()
-        n = 10
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for _ in range(n):
             step()
         e1.record(stream)
         stream.synchronize()
-    ms = e0.elapsed_time(e1) / n
-    flops = 2 * 3 * s.d * s.f * T * s.k + 2 * 3 * s.d * s.f_shared * T + 2 * T * s.E * s.d
-    del D
-    return {"workload": "prefill T=%d, same layer, router bias N(0,1)" % T, "tokens_per_s": T / (ms / 1e3),
-            "ms_per_step": ms, "tflops": flops / (ms / 1e3) / 1e12,
-            "frac_of_bf16_peak": flops / (ms / 1e3) / 1e12 / tf, "peak_tflops": tf, "peak_kind": peak_kind}
+    return e0.elapsed_time(e1) / n
 
 
 class StepTimer:
@@ -509,21 +547,13 @@ def run_workloads(ds4moe, torch, stream, hbm, tf, peak_kind):
         T = wl.tokens[0]
         D = ds4moe.DeviceLayer(synth.make_layer(wl), max_tokens=T)
         x = torch.from_numpy(synth.activations(wl, T)).cuda().view(torch.bfloat16)
-        with torch.cuda.stream(stream):
-            for _ in range(2):
-                D.forward_grouped(x)
-            stream.synchronize()
-            n = 5
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            for _ in range(n):
-                D.forward_grouped(x)
-            e1.record(stream)
-            stream.synchronize()
-        ms = e0.elapsed_time(e1) / n
         flops = 2 * 3 * s.d * s.f * T * s.k + 2 * 3 * s.d * s.f_shared * T + 2 * T * s.E * s.d
-        prefill = {"T": T, "tokens_per_s": T / (ms / 1e3), "ms_per_step": ms, "tflops": flops / (ms / 1e3) / 1e12,
-                   "frac_of_bf16_peak": flops / (ms / 1e3) / 1e12 / tf}
+        prefill = {"T": T}
+        for name, step in (("deterministic", lambda: D.forward_grouped(x)), ("fused", lambda: D.forward_fused(x))):
+            ms = device_ms(torch, stream, step, warmup=2, n=5)
+            assert ds4moe.last_device_error() == 0
+            prefill[name] = {"tokens_per_s": T / (ms / 1e3), "ms_per_step": ms, "tflops": flops / (ms / 1e3) / 1e12,
+                             "frac_of_bf16_peak": flops / (ms / 1e3) / 1e12 / tf}
         del x
         n = 32
         x1 = torch.from_numpy(synth.activations(wl, n, stream=1)).cuda().view(torch.bfloat16)
@@ -545,32 +575,37 @@ def run_workloads(ds4moe, torch, stream, hbm, tf, peak_kind):
 
 def run_profile_case(args):
     """Small case for ncu captures, same kernels and shapes as the benchmark but fewer experts resident:
-    decode layer d=4096, f=2048, k=8, shared 2048 with E=16 experts (the 8 a token uses stream 56 MB of packed
-    weights + 50 MB of shared weights per pass, more than L2), 16 eager B=1 passes; optionally a prefill of
-    T tokens on E=64 experts (T=1024, k=8 keeps the prefill workload's 128 tokens per expert on average)."""
+    the decode layer d=4096, f=2048, k=8, shared 2048 (IQ2X/Q2K, or Q4K throughout with --profile-layer q4) with
+    E=16 experts (the 8 a token uses stream 56 MB of packed IQ2X/Q2K weights, 118 MB of Q4K, + 50 MB of shared
+    weights per pass, about L2's size or more), 16 eager decode steps of --profile-batch tokens each; optionally
+    a prefill of T tokens on E=64 experts (T=1024, k=8 keeps the prefill workload's 128 tokens per expert on
+    average), in the deterministic and the fused-combine form."""
     import dataclasses
 
     import torch
     from bit_quantized_moe_02_b200 import ds4moe
-    base = synth.WORKLOADS["decode"]
+    base = synth.WORKLOADS["decode" if args.profile_layer == "decode" else "q4"]
     wl = dataclasses.replace(base, shape=dataclasses.replace(base.shape, E=16))
-    D = ds4moe.DeviceLayer(synth.make_layer(wl), max_tokens=1)
-    xs = torch.from_numpy(synth.activations(wl, 16, stream=3)).cuda().view(torch.bfloat16)
+    B = args.profile_batch
+    D = ds4moe.DeviceLayer(synth.make_layer(wl), max_tokens=B)
+    xs = torch.from_numpy(synth.activations(wl, 16 * B, stream=3)).cuda().view(torch.bfloat16)
     for i in range(16):
-        D.forward(xs[i:i + 1])
+        D.forward(xs[i * B:(i + 1) * B])
     torch.cuda.synchronize()
     if args.profile_prefill:
         del D
-        pb = synth.WORKLOADS["prefill"]
+        pb = synth.WORKLOADS["prefill" if args.profile_layer == "decode" else "q4"]
         wlp = dataclasses.replace(pb, shape=dataclasses.replace(pb.shape, E=64))
         T = args.profile_prefill
         P = ds4moe.DeviceLayer(synth.make_layer(wlp), max_tokens=T)
         x = torch.from_numpy(synth.activations(wlp, T)).cuda().view(torch.bfloat16)
         for _ in range(2):
             P.forward_grouped(x)
+            P.forward_fused(x)
         torch.cuda.synchronize()
     assert ds4moe.last_device_error() == 0
-    print(json.dumps({"profile_case": "ok", "prefill_T": args.profile_prefill}))
+    print(json.dumps({"profile_case": "ok", "layer": args.profile_layer, "batch": B,
+                      "prefill_T": args.profile_prefill}))
 
 
 def main():
@@ -584,6 +619,9 @@ def main():
     ap.add_argument("--no-workloads", action="store_true", help="skip the tiny / batched / q4 measurements")
     ap.add_argument("--profile-case", action="store_true", help="small case for ncu captures (see profiles/)")
     ap.add_argument("--profile-prefill", type=int, default=0, help="with --profile-case: also run a T-token prefill")
+    ap.add_argument("--profile-layer", default="decode", choices=["decode", "q4"],
+                    help="with --profile-case: IQ2X/Q2K decode layer or its Q4K variant")
+    ap.add_argument("--profile-batch", type=int, default=1, help="with --profile-case: tokens per decode step")
     args = ap.parse_args()
     if args.profile_case:
         run_profile_case(args)

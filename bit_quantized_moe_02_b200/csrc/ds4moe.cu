@@ -208,8 +208,9 @@ DecodeWs decode_ws(const ds4moe_experts *ex, int k) {
 
 struct GroupedWs {
     uint64_t x16, xinv, blk, counts, offsets, tile_e, tile_pos0, tile_cnt, meta, perm_tok, perm_w, x_perm, h16, hexp, hs;
-    uint64_t y_perm, inv, y_shared;  // only used when decode B > 1 runs through the grouped path
-    uint64_t total_grouped, total_decode;
+    uint64_t inv;                    // inverse map of the fused-combine call (the caller's buffer otherwise)
+    uint64_t y_perm, y_shared;       // only used when decode B > 16 runs through the grouped path
+    uint64_t total_grouped, total_fused, total_decode;
     int nblk, max_tiles;
 };
 GroupedWs grouped_ws(const ds4moe_experts *ex, int T, int k) {
@@ -239,8 +240,9 @@ GroupedWs grouped_ws(const ds4moe_experts *ex, int T, int k) {
     w.hexp = take(uint64_t(w.max_tiles) * (ex->f / tc::M) * 4);  // fp16 h exponent per (token tile, row tile)
     w.hs = take(uint64_t(T) * (ex->f_shared > 0 ? ex->f_shared : 1) * 2);
     w.total_grouped = o;
-    w.y_perm = take(N * ex->d * 4);
     w.inv = take(N * 4);
+    w.total_fused = o;
+    w.y_perm = take(N * ex->d * 4);
     w.y_shared = take(uint64_t(T) * ex->d * 4);
     w.total_decode = o;
     return w;
@@ -287,8 +289,12 @@ ds4moe_status launch_grouped(const GroupedArgs &ga, int row_units, int col_tiles
     return DS4MOE_OK;
 }
 
+// fused_out == NULL: routed rows to y_perm (position order) and the shared expert to y_shared, for ds4moe_combine.
+// fused_out != NULL: the shared expert's output is stored into fused_out first (zeros without one), then the
+// routed down GEMM adds each weighted row into its token's row of fused_out (y_perm, y_shared unused).
 ds4moe_status run_grouped(const ds4moe_experts *ex, const void *x, int T, const int32_t *ids, const float *weights,
-                          int k, float *y_perm, int32_t *inv_perm, float *y_shared, uint8_t *ws, cudaStream_t st) {
+                          int k, float *y_perm, int32_t *inv_perm, float *y_shared, uint8_t *ws, cudaStream_t st,
+                          float *fused_out = nullptr) {
     const GroupedWs W = grouped_ws(ex, T, k);
     const ExpertsDev D = to_dev(ex);
     const int N = T * k;
@@ -324,6 +330,28 @@ ds4moe_status run_grouped(const ds4moe_experts *ex, const void *x, int T, const 
     gather_rows_kernel<<<(N + 7) / 8, 256, 0, st>>>(x16, ex->d, perm_tok, N, x_perm);
     DS4_CHECK_LAUNCH();
 
+    auto shared_expert = [&](float *dst) -> ds4moe_status {
+        const int ct = (T + tile_n - 1) / tile_n;
+        // Shared expert, a dense bf16 SwiGLU: A and the tokens both come by TMA as bf16 (x as given, hs written
+        // as bf16)
+        GroupedArgs s1 = {};
+        s1.a0 = static_cast<const uint8_t *>(ex->sh_gate); s1.a1 = static_cast<const uint8_t *>(ex->sh_up);
+        s1.a_stride = 0; s1.rows = ex->f_shared; s1.K = ex->d;
+        s1.b_src = x16; s1.b_colscale = nullptr; s1.n_pos = T; s1.out = hs; s1.ldo = ex->f_shared;
+        const ds4moe_status r = launch_grouped<tc::FMT_BF16D, true>(s1, ex->f_shared, ct, xb, T, st);
+        if (r != DS4MOE_OK) return r;
+        GroupedArgs s2 = {};
+        s2.a0 = static_cast<const uint8_t *>(ex->sh_down); s2.a_stride = 0; s2.rows = ex->d; s2.K = ex->f_shared;
+        s2.b_src = hs; s2.n_pos = T; s2.out = dst; s2.ldo = ex->d;
+        return launch_grouped<tc::FMT_BF16D, false>(s2, ex->d, ct, hs, T, st);
+    };
+    ds4moe_status s;
+    if (fused_out) {  // the shared expert's rows (or zeros) first: the routed rows are added on top
+        if (ex->f_shared > 0) s = shared_expert(fused_out);
+        else s = cudaMemsetAsync(fused_out, 0, size_t(T) * ex->d * 4, st) == cudaSuccess ? DS4MOE_OK : DS4MOE_ECUDA;
+        if (s != DS4MOE_OK) return s;
+    }
+
     // routed GEMM-1: gate/up -> h16
     GroupedArgs g1 = {};
     g1.a0 = D.gate; g1.a1 = D.up; g1.a_stride = D.gate_stride; g1.a1_stride = D.up_stride; g1.pa = D.pg;
@@ -332,7 +360,6 @@ ds4moe_status run_grouped(const ds4moe_experts *ex, const void *x, int T, const 
     g1.b_src = x16; g1.b_rowidx = perm_tok; g1.b_colscale = xinv;
     g1.tile_e = tile_e; g1.tile_pos0 = tile_pos0; g1.tile_cnt = tile_cnt; g1.n_tiles = meta;
     g1.out = h16; g1.ldo = ex->f; g1.h_exp_out = hexp;
-    ds4moe_status s;
     if (ex->fmt_gate == DS4MOE_FMT_IQ2X) s = launch_grouped<DS4MOE_FMT_IQ2X, true>(g1, ex->f, W.max_tiles, x_perm, N, st);
     else s = launch_grouped<DS4MOE_FMT_Q4K, true>(g1, ex->f, W.max_tiles, x_perm, N, st);
     if (s != DS4MOE_OK) return s;
@@ -342,27 +369,13 @@ ds4moe_status run_grouped(const ds4moe_experts *ex, const void *x, int T, const 
     g2.a0 = D.down; g2.a_stride = D.down_stride; g2.pa = D.pd; g2.rows = ex->d; g2.K = ex->f; g2.n_mats = ex->E;
     g2.b_src = h16; g2.b_rowidx = nullptr; g2.b_colscale = nullptr;
     g2.tile_e = tile_e; g2.tile_pos0 = tile_pos0; g2.tile_cnt = tile_cnt; g2.n_tiles = meta;
-    g2.pos_weight = perm_w; g2.out = y_perm; g2.ldo = ex->d; g2.h_exp_in = hexp;
+    g2.pos_weight = perm_w; g2.out = fused_out ? fused_out : y_perm; g2.ldo = ex->d; g2.h_exp_in = hexp;
+    g2.out_row = fused_out ? perm_tok : nullptr;
     if (ex->fmt_down == DS4MOE_FMT_Q2K) s = launch_grouped<DS4MOE_FMT_Q2K, false>(g2, ex->d, W.max_tiles, h16, N, st);
     else s = launch_grouped<DS4MOE_FMT_Q4K, false>(g2, ex->d, W.max_tiles, h16, N, st);
     if (s != DS4MOE_OK) return s;
+    if (!fused_out && ex->f_shared > 0) return shared_expert(y_shared);
 
-    if (ex->f_shared > 0) {
-        const int ct = (T + tile_n - 1) / tile_n;
-        // Shared expert, a dense bf16 SwiGLU: A and the tokens both come by TMA as bf16 (x as given, hs written
-        // as bf16)
-        GroupedArgs s1 = {};
-        s1.a0 = static_cast<const uint8_t *>(ex->sh_gate); s1.a1 = static_cast<const uint8_t *>(ex->sh_up);
-        s1.a_stride = 0; s1.rows = ex->f_shared; s1.K = ex->d;
-        s1.b_src = x16; s1.b_colscale = nullptr; s1.n_pos = T; s1.out = hs; s1.ldo = ex->f_shared;
-        s = launch_grouped<tc::FMT_BF16D, true>(s1, ex->f_shared, ct, xb, T, st);
-        if (s != DS4MOE_OK) return s;
-        GroupedArgs s2 = {};
-        s2.a0 = static_cast<const uint8_t *>(ex->sh_down); s2.a_stride = 0; s2.rows = ex->d; s2.K = ex->f_shared;
-        s2.b_src = hs; s2.n_pos = T; s2.out = y_shared; s2.ldo = ex->d;
-        s = launch_grouped<tc::FMT_BF16D, false>(s2, ex->d, ct, hs, T, st);
-        if (s != DS4MOE_OK) return s;
-    }
     return DS4MOE_OK;
 }
 
@@ -698,6 +711,24 @@ ds4moe_status ds4moe_expert_ffn_grouped(const ds4moe_experts *ex, const void *x_
     if (ws_bytes < grouped_ws(ex, T, k).total_grouped) return DS4MOE_ENOWORKSPACE;
     return run_grouped(ex, x_bf16, T, ids, weights, k, y_perm, inv_perm, ex->f_shared > 0 ? y_shared : nullptr,
                        static_cast<uint8_t *>(ws), cs(stream));
+}
+
+ds4moe_status ds4moe_expert_ffn_grouped_fused(const ds4moe_experts *ex, const void *x_bf16, int T, const int32_t *ids,
+                                              const float *weights, int k, float *out, void *ws, size_t ws_bytes,
+                                              ds4moe_stream stream) {
+    (void)cudaGetLastError();  // report only errors raised by this call's launches
+    ds4moe_status s = check_experts(ex);
+    if (s != DS4MOE_OK) return s;
+    if (T < 0 || k < 1 || k > ex->E || ex->E > MAX_E_GROUPED) return DS4MOE_EINVAL;
+    if (!grouped_supported(ex)) return DS4MOE_EUNSUPPORTED;
+    if (T == 0) return DS4MOE_OK;
+    if (!x_bf16 || !ids || !weights || !out || !ws || !aligned16(x_bf16) || !aligned256(ws) || !aligned16(out))
+        return DS4MOE_EINVAL;
+    const GroupedWs W = grouped_ws(ex, T, k);
+    if (ws_bytes < W.total_fused) return DS4MOE_ENOWORKSPACE;
+    uint8_t *w8 = static_cast<uint8_t *>(ws);
+    return run_grouped(ex, x_bf16, T, ids, weights, k, nullptr, reinterpret_cast<int32_t *>(w8 + W.inv), nullptr, w8,
+                       cs(stream), out);
 }
 
 ds4moe_status ds4moe_combine(const float *y_perm, const int32_t *inv_perm, const float *y_shared, int T, int d, int k,

@@ -32,6 +32,9 @@ struct GroupedArgs {
     // product, and the result, is unchanged.  NULL: no scaling.
     int32_t *h_exp_out;
     const int32_t *h_exp_in;
+    // DOWN: when set, row p of the result is added (red.global.add) into out row out_row[p] instead of being
+    // stored at row p: the weighted combine of the layer fused into the epilogue
+    const int32_t *out_row;
 };
 
 // 128-byte swizzle of a K-major fp16 tile: 16-byte chunk `chunk` of row `row`

@@ -158,16 +158,19 @@ __device__ __forceinline__ void mma_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
 }
 
+// The wait sits in the same asm statement as the load: the registers are undefined until tcgen05.wait::ld, and
+// outputs of a separate statement would let the compiler schedule their uses before the wait.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,"
-        "%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        "%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
         : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
           "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
           "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
           "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+        : "r"(taddr)
+        : "memory");
 }
 
 // 2D TMA tensor load (tile mode, no multicast): box at (c0 = inner element, c1 = row) into shared memory,
@@ -374,6 +377,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
     __shared__ float s_colsc[NT];
+    __shared__ int s_orow[NT];      // DOWN with a fused combine: output row (token) of each position
     __shared__ uint32_t s_hmax;     // GATEUP: largest |h| of the tile (float bits; non-finite sorts above +inf)
     __shared__ float s_hsc[MAX_K / 128];  // DOWN: weight factor 2^e of each 128-wide K range
 
@@ -403,14 +407,14 @@ __global__ void __launch_bounds__(THREADS, 1)
 
     if (tid == 0) {
         for (int s = 0; s < S; s++) {
-            mbar_init(full_a(s), N_WA);
+            mbar_init(full_a(s), N_WA * 32);  // every producer thread arrives (see the producers)
             mbar_init(full_b(s), 1);
             mbar_init(empty(s), 1);
         }
         mbar_init(accum_bar, 1);
         for (int s = 0; s < 2; s++) {
             mbar_init(full_p(s), 1);
-            mbar_init(empty_p(s), N_WA);
+            mbar_init(empty_p(s), N_WA * 32);
         }
         s_abort = 0;
         s_hmax = 0;
@@ -429,6 +433,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             const int pos = pos0 + tid;
             if (a.b_colscale) sc *= a.b_colscale[a.b_rowidx ? a.b_rowidx[pos] : pos];
             if (a.pos_weight) sc *= a.pos_weight[pos];
+            if (a.out_row) s_orow[tid] = a.out_row[pos];
         }
         s_colsc[tid] = sc;
     }
@@ -579,8 +584,11 @@ __global__ void __launch_bounds__(THREADS, 1)
                     cur.w[8] = sc.x; cur.w[9] = sc.y; cur.w[10] = sc.z; cur.w[11] = sc.w;
                     cur.w[12] = s00;
                 }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(empty_p(sl));  // the slot may be refilled
+                // The slot is refilled by TMA (async proxy) as soon as every thread has arrived, and the words
+                // just loaded are used only later: the proxy fence orders this thread's shared-memory reads
+                // before that copy (without it, the last thread to arrive could see the next block's bytes).
+                fence_proxy_async();
+                mbar_arrive(empty_p(sl));
                 s00 = s10; s01 = s11; s10 = s20; s11 = s21;
 #pragma unroll
                 for (int jj = 0; jj < 4; jj++) {
@@ -601,9 +609,10 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
                     for (int c = 0; c < NOUT; c++)
                         *reinterpret_cast<uint4 *>(ast + swz(R, (GATEUP ? 0 : h * 4) + c)) = o[c];
+                    // each writing thread makes its own stores visible to the tensor core (async proxy) and
+                    // releases them itself
                     fence_proxy_async();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(full_a(s));
+                    mbar_arrive(full_a(s));
                 }
             }
             if (inf) set_device_error(DS4MOE_EDEVICE);
@@ -660,8 +669,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                         for (int c = 0; c < NOUT; c++)
                             *reinterpret_cast<uint4 *>(ast + swz(R, (GATEUP ? 0 : h * 4) + c)) = o[c];
                         fence_proxy_async();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(full_a(s));
+                        mbar_arrive(full_a(s));
                     }
                 }
             }
@@ -724,10 +732,23 @@ __global__ void __launch_bounds__(THREADS, 1)
                     for (int c0 = 0; c0 < n_eff; c0 += 32) {
                         uint32_t g[32];
                         tmem_ld32(tq + c0, g);
+                        if (a.out_row) {
+                            // fused combine: each warp adds 32 consecutive rows of one token (coalesced reductions)
 #pragma unroll
-                        for (int i = 0; i < 32; i++) {
-                            const int n = c0 + i;
-                            if (n < cnt) out[size_t(pos0 + n) * a.ldo + blockIdx.x * M + r] = __uint_as_float(g[i]) * s_colsc[n];
+                            for (int i = 0; i < 32; i++) {
+                                const int n = c0 + i;
+                                if (n < cnt) {
+                                    float *dst = out + size_t(s_orow[n]) * a.ldo + blockIdx.x * M + r;
+                                    const float v = __uint_as_float(g[i]) * s_colsc[n];
+                                    asm volatile("red.global.add.f32 [%0], %1;" ::"l"(dst), "f"(v) : "memory");
+                                }
+                            }
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 32; i++) {
+                                const int n = c0 + i;
+                                if (n < cnt) out[size_t(pos0 + n) * a.ldo + blockIdx.x * M + r] = __uint_as_float(g[i]) * s_colsc[n];
+                            }
                         }
                     }
                 }

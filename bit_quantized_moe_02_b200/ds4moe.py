@@ -28,7 +28,8 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported", 3: "CUDA error", 4: 
 EXPORTS = ["ds4moe_status_string", "ds4moe_prepared_bytes", "ds4moe_prepare", "ds4moe_dequant",
            "ds4moe_route_workspace_size", "ds4moe_route", "ds4moe_workspace_size", "ds4moe_expert_ffn_decode",
            "ds4moe_expert_ffn_grouped", "ds4moe_combine", "ds4moe_last_device_error", "ds4moe_decode_gateup",
-           "ds4moe_decode_down", "ds4moe_expert_ffn_decode_noalloc", "ds4moe_selftest_wait_timeout"]
+           "ds4moe_decode_down", "ds4moe_expert_ffn_decode_noalloc", "ds4moe_selftest_wait_timeout",
+           "ds4moe_expert_ffn_grouped_fused"]
 
 
 class Ds4moeError(RuntimeError):
@@ -71,6 +72,7 @@ def lib():
         l.ds4moe_expert_ffn_decode.argtypes = [ctypes.POINTER(Experts), vp, i32, vp, vp, i32, vp, vp, sz, vp]
         l.ds4moe_expert_ffn_grouped.argtypes = [ctypes.POINTER(Experts), vp, i32, vp, vp, i32, vp, vp, vp, vp, sz,
                                                 vp]
+        l.ds4moe_expert_ffn_grouped_fused.argtypes = [ctypes.POINTER(Experts), vp, i32, vp, vp, i32, vp, vp, sz, vp]
         l.ds4moe_combine.argtypes = [vp, vp, vp, i32, i32, i32, vp, vp]
         l.ds4moe_last_device_error.argtypes = [vp, ctypes.POINTER(ctypes.c_int32)]
         l.ds4moe_decode_gateup.argtypes = [ctypes.POINTER(Experts), vp, vp, i32, vp, sz, vp]
@@ -239,6 +241,22 @@ def expert_ffn_grouped(ex: Experts, x: torch.Tensor, ids: torch.Tensor, weights:
                                            _stream()), "expert_ffn_grouped")
 
 
+def expert_ffn_grouped_fused(ex: Experts, x: torch.Tensor, ids: torch.Tensor, weights: torch.Tensor,
+                             ws: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Prefill with the combine fused into the down GEMM: returns the layer output [T, d] (fp32)."""
+    T, k = ids.shape
+    out = torch.empty((T, ex.d), dtype=torch.float32, device=x.device) if out is None else out
+    dev = _cur()
+    px = _arg(x, "expert_ffn_grouped_fused: x", dev, 2, shape=(T, ex.d))
+    pi = _arg(ids, "expert_ffn_grouped_fused: ids", dev, 4)
+    pr = _arg(weights, "expert_ffn_grouped_fused: weights", dev, 4, shape=(T, k))
+    po = _arg(out, "expert_ffn_grouped_fused: out", dev, 4, numel=T * ex.d)
+    ps = _arg(ws, "expert_ffn_grouped_fused: workspace", dev, ws.element_size())
+    _check(lib().ds4moe_expert_ffn_grouped_fused(ctypes.byref(ex), px, T, pi, pr, k, po, ps, _bytes(ws),
+                                                 _stream()), "expert_ffn_grouped_fused")
+    return out
+
+
 def combine(y_perm: torch.Tensor, inv_perm: torch.Tensor, y_shared: Optional[torch.Tensor], T: int, d: int, k: int,
             out: Optional[torch.Tensor] = None) -> torch.Tensor:
     out = torch.empty((T, d), dtype=torch.float32, device=y_perm.device) if out is None else out
@@ -348,6 +366,15 @@ class DeviceLayer:
         expert_ffn_grouped(self.ex, x, ids, w, self.ws, y_perm, inv, ys)
         out = combine(y_perm, inv, ys, T, s.d, s.k)
         return out, ids, w, y_perm, inv
+
+    def forward_fused(self, x: torch.Tensor, out: Optional[torch.Tensor] = None):
+        """Prefill entry with the combine fused into the down GEMM (returns out, ids, weights).  The k routed
+        rows of a token are summed by atomic adds, in no fixed order."""
+        T = x.shape[0]
+        self.reserve(T)
+        ids, w = self.route(x, ids=self.ids_buf[:T], weights=self.w_buf[:T])
+        out = expert_ffn_grouped_fused(self.ex, x, ids, w, self.ws, out=out)
+        return out, ids, w
 
 
 class DecodeGraph:

@@ -275,6 +275,23 @@ ds4moe_status ds4moe_expert_ffn_grouped(const ds4moe_experts *ex, const void *x_
                                         const float *weights, int k, float *y_perm, int32_t *inv_perm,
                                         float *y_shared, void *ws, size_t ws_bytes, ds4moe_stream stream);
 
+/* Prefill with the combine fused into the routed down GEMM: out[T x d] (fp32)
+ * = the full layer output, with no y_perm, inv_perm or y_shared.  The shared
+ * expert's output is stored into out first (zeros when the layer has none);
+ * the routed down GEMM's epilogue then adds each weighted row w_(t,j) y_(t,j)
+ * straight into out[t] with fp32 atomic adds.  The k additions to a row come
+ * from different CTAs in no fixed order, so results agree with
+ * ds4moe_expert_ffn_grouped + ds4moe_combine only up to fp32 rounding of the
+ * summation order and may differ in the last bits from run to run.  Same
+ * limits and h scaling as ds4moe_expert_ffn_grouped; out is 16-byte aligned
+ * and must not overlap x or the workspace; the workspace may be smaller
+ * (ds4moe_workspace_size is enough).  Passage: the weighted combine of the
+ * expert outputs in the layer formula at the top of this file (ds4 news
+ * summary, "model weights"); the pages fix no summation order. */
+ds4moe_status ds4moe_expert_ffn_grouped_fused(const ds4moe_experts *ex, const void *x_bf16, int T,
+                                              const int32_t *ids, const float *weights, int k, float *out, void *ws,
+                                              size_t ws_bytes, ds4moe_stream stream);
+
 /* out[t] = y_shared[t] + sum_{j<k} y_perm[inv_perm[t*k+j]] (j in increasing
  * order, fp32).  y_shared may be NULL.  d multiple of 4.  This is the last
  * line of the layer formula at the top of this file; the pages fix no

@@ -76,6 +76,12 @@ def test_host_side_argument_checks():
     bad.f_shared = 256  # shared expert without weights
     assert lib.ds4moe_expert_ffn_grouped(ctypes.byref(bad), fake, 4, fake, fake, 2, fake, fake, None, fake, 1 << 30,
                                          None) == 1
+    # fused-combine prefill: missing output, misaligned output, short workspace
+    assert lib.ds4moe_expert_ffn_grouped_fused(ctypes.byref(ex), fake, 4, fake, fake, 2, None, fake, 1 << 30,
+                                               None) == 1
+    assert lib.ds4moe_expert_ffn_grouped_fused(ctypes.byref(ex), fake, 4, fake, fake, 2, ctypes.c_void_p((1 << 20) + 4),
+                                               fake, 1 << 30, None) == 1
+    assert lib.ds4moe_expert_ffn_grouped_fused(ctypes.byref(ex), fake, 4, fake, fake, 2, fake, fake, 16, None) == 4
     assert lib.ds4moe_last_device_error(None, None) == 1
 
 
@@ -120,6 +126,8 @@ def test_grouped_path_expert_limit():
     assert lib.ds4moe_workspace_size(ctypes.byref(big), 16, 2) > 0
     assert lib.ds4moe_expert_ffn_grouped(ctypes.byref(big), fake, 4, fake, fake, 2, fake, fake, None, fake,
                                          1 << 30, None) == 1
+    assert lib.ds4moe_expert_ffn_grouped_fused(ctypes.byref(big), fake, 4, fake, fake, 2, fake, fake, 1 << 30,
+                                               None) == 1
     assert lib.ds4moe_expert_ffn_decode(ctypes.byref(big), fake, 17, fake, fake, 2, fake, fake, 1 << 30, None) == 1
     mixed = ds4moe.Experts(256, 512, 2048, 0, 2, 2, 1, 1 << 20, 1 << 21, 1 << 22, 1 << 17, 1 << 17, 1 << 17, None,
                            None, None, None)  # Q4K gate/up with Q2K down: even B = 1 needs the grouped path
@@ -137,9 +145,12 @@ def test_empty_inputs_are_no_ops():
     assert lib.ds4moe_expert_ffn_decode(ctypes.byref(ex), None, 0, None, None, 2, None, None, 0, None) == 0
     assert lib.ds4moe_expert_ffn_grouped(ctypes.byref(ex), None, 0, None, None, 2, None, None, None, None, 0,
                                          None) == 0
+    assert lib.ds4moe_expert_ffn_grouped_fused(ctypes.byref(ex), None, 0, None, None, 2, None, None, 0, None) == 0
     assert lib.ds4moe_combine(None, None, None, 0, 256, 2, None, None) == 0
     # negative counts are errors, not no-ops
     assert lib.ds4moe_expert_ffn_decode(ctypes.byref(ex), None, -1, None, None, 2, None, None, 0, None) == 1
     assert lib.ds4moe_expert_ffn_grouped(ctypes.byref(ex), None, -1, None, None, 2, None, None, None, None, 0,
                                          None) == 1
+    assert lib.ds4moe_expert_ffn_grouped_fused(ctypes.byref(ex), None, -1, None, None, 2, None, None, 0,
+                                               None) == 1
     assert lib.ds4moe_combine(None, None, None, -1, 256, 2, None, None) == 1

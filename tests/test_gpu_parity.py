@@ -113,6 +113,8 @@ def run_and_compare(ds4, L, x, path, nthreads=None):
         out, ids = torch.cat(outs), torch.cat(idss)
     elif path == "batched":
         out, ids, _ = D.forward(xt, return_routing=True)
+    elif path == "fused":
+        out, ids, _ = D.forward_fused(xt)
     else:
         out, ids, _, _, _ = D.forward_grouped(xt)
     torch.cuda.synchronize()
@@ -130,11 +132,36 @@ def test_tiny_decode(ds4):
     run_and_compare(ds4, L, x, "decode")
 
 
-def test_tiny_grouped(ds4):
+@pytest.mark.parametrize("path", ["grouped", "fused"])
+def test_tiny_grouped(ds4, path):
     wl = synth.WORKLOADS["tiny"]
     L = synth.make_layer(wl)
     x = synth.activations(wl, 150)
-    run_and_compare(ds4, L, x, "grouped")
+    run_and_compare(ds4, L, x, path)
+
+
+@pytest.mark.parametrize("fs", [512, 0])
+def test_fused_combine_matches_deterministic(ds4, fs):
+    """The fused-combine prefill adds the k weighted rows of a token by atomic adds; it must agree with the
+    deterministic grouped + combine path up to fp32 summation order (with and without a shared expert, whose
+    absence makes the fused call zero the output first), and with the oracle at the layer tolerance."""
+    shape = synth.LayerShape(d=1024, E=16, f=768, k=6, f_shared=fs)
+    L = layer_of(shape, 1.0, 91 + fs)
+    x = synth.f32_to_bf16_bits(synth.rng(9, fs).normal(size=(300, shape.d)).astype(np.float32))
+    D = ds4.DeviceLayer(L, max_tokens=x.shape[0])
+    xt = dev(x).view(torch.bfloat16)
+    ref_out, ref_ids, ref_w, _, _ = D.forward_grouped(xt)
+    out = torch.full((x.shape[0], shape.d), float("nan"), dtype=torch.float32, device="cuda")
+    got, ids, w = D.forward_fused(xt, out=out)
+    torch.cuda.synchronize()
+    assert ds4.last_device_error() == 0
+    assert got.data_ptr() == out.data_ptr()
+    assert torch.equal(ids, ref_ids) and torch.equal(w, ref_w)
+    a, b = got.double().cpu().numpy(), ref_out.double().cpu().numpy()
+    assert np.all(np.isfinite(a))
+    # k + 1 fp32 terms per element: reordering moves the sum by a few ulps of the largest partial sum
+    assert np.max(np.abs(a - b)) <= 1e-5 * np.max(np.abs(b))
+    run_and_compare(ds4, L, x, "fused")
 
 
 @pytest.mark.parametrize("d,f,fs,E,k", [(512, 1024, 512, 16, 4), (1024, 256, 0, 12, 3), (2048, 512, 256, 32, 8)])
@@ -144,6 +171,7 @@ def test_mid_shapes_decode_and_grouped(ds4, d, f, fs, E, k):
     x = synth.f32_to_bf16_bits(synth.rng(3, d, f).normal(size=(200, d)).astype(np.float32))
     run_and_compare(ds4, L, x[:4], "decode")
     run_and_compare(ds4, L, x, "grouped")  # several token tiles, ragged tail
+    run_and_compare(ds4, L, x, "fused")
 
 
 @pytest.mark.parametrize("d,f,fs,E,k", [(2048, 512, 1024, 16, 4), (4096, 1024, 2048, 16, 8)])
@@ -171,6 +199,7 @@ def test_q4k_layer_small(ds4):
     L = layer_of(shape, 1.0, 77)
     x = synth.f32_to_bf16_bits(synth.rng(4).normal(size=(70, 512)).astype(np.float32))
     run_and_compare(ds4, L, x, "grouped")
+    run_and_compare(ds4, L, x, "fused")
     run_and_compare(ds4, L, x[:2], "decode")
 
 

@@ -80,6 +80,8 @@ def compare(ds4, L, x, path):
             outs.append(o)
             idss.append(ids)
         out, ids = torch.cat(outs), torch.cat(idss)
+    elif path == "fused":
+        out, ids, _ = D.forward_fused(xt)
     else:
         out, ids, _, _, _ = D.forward_grouped(xt)
     torch.cuda.synchronize()
@@ -114,7 +116,8 @@ def test_decode_q2k_sub_blocks_at_their_bound(ds4):
     compare(ds4, L, x, "decode")
 
 
-def test_grouped_swiglu_output_beyond_fp16(ds4):
+@pytest.mark.parametrize("path", ["grouped", "fused"])
+def test_grouped_swiglu_output_beyond_fp16(ds4, path):
     """Block scales d = 0.25 make |h| reach about 1e8 (far beyond fp16): the grouped path scales the stored h by a
     power of two per token tile and row block and the down GEMM multiplies the weights back."""
     shape = synth.LayerShape(d=512, E=8, f=512, k=2, f_shared=256)
@@ -131,7 +134,7 @@ def test_grouped_swiglu_output_beyond_fp16(ds4):
     L.expert = big
     L.drop_cache = lambda: None
     x = synth.f32_to_bf16_bits(synth.rng(64).normal(0, 4.0, size=(150, shape.d)).astype(np.float32))
-    rel, mx = compare(ds4, L, x, "grouped")
+    rel, mx = compare(ds4, L, x, path)
     ref = parity.oracle_layer(L, x[:4])
     assert np.abs(ref["out"]).max() > 1e6  # the case really is beyond the fp16 range
 
