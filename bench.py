@@ -224,7 +224,7 @@ def run_reference(args, ws, rank):
 # our arm
 
 
-GATEUP_KERNEL = "decode_gateup_kernel<8, 4>"
+GATEUP_KERNEL = "decode_gateup_kernel<0, 8, 4>"
 GATEUP_SRC = os.path.join(ROOT, "bit_quantized_moe_02_b200", "csrc", "decode_gemv.cuh")
 
 
