@@ -17,10 +17,20 @@
 //               256-wide K block at a time, with 3D TMA copies into a 2-slot
 //               shared-memory ring (Q4K and bf16 producers load into registers).
 //   warps 4-11  dequantize the packed blocks in registers (shared-memory
-//               codebook / sign-bit XOR / fp16 scale) and write fp16 tiles in
-//               the same swizzled K-major layout the MMA descriptor describes.
-//               Warps 4-7 then run the epilogue: tcgen05.ld the accumulators,
-//               SwiGLU (gate/up) or routing-weight scaling (down), stores.
+//               codebook / sign-bit XOR / fp16 scale) and hand the fp16 A
+//               tiles to the MMA: for the IQ2X gate/up and the packed down
+//               kernels they go to tensor memory (tcgen05.st, row = TMEM
+//               lane) and the MMA reads A from there, which keeps them out of
+//               shared memory (the MMA's operand reads and the producers'
+//               stores share its bandwidth); the Q4K gate/up kernel writes
+//               them to shared memory in the swizzled K-major layout the MMA
+//               descriptor describes.  Warps 4-7 then run the epilogue:
+//               tcgen05.ld the accumulators, SwiGLU (gate/up) or
+//               routing-weight scaling (down), stores.
+//
+// The packed down kernels need 256 TMEM columns and ~90 KB of shared memory,
+// so two CTAs share an SM and one's prologue and epilogue overlap the other's
+// main loop.
 //
 // Gate and up share one work item: two accumulators (TMEM columns [0,128) and
 // [128,256)) hold matching rows, so each epilogue thread owns a gate/up pair.
@@ -68,12 +78,23 @@ struct PackTma {
 
 template <int AFMT, bool GATEUP>
 struct Cfg {
-    static constexpr int STAGES = (AFMT == DS4MOE_FMT_IQ2X && GATEUP) ? 3 : 4;
-    static constexpr int STAGE = (GATEUP ? 2 : 1) * A_TILE + B_TILE;
-    static constexpr int TMEM_COLS = GATEUP ? 256 : 128;
+    // ATM: the dequantized A tiles live in tensor memory (tcgen05.st by the producers, MMA with A from TMEM);
+    // the shared-memory stages then hold only the token tile
+    static constexpr bool ATM = (AFMT == DS4MOE_FMT_IQ2X && GATEUP) || (!is_dense<AFMT>() && !GATEUP);
+    // the packed down kernels then fit twice per SM (shared memory, TMEM, registers), so one CTA's prologue and
+    // epilogue overlap the other's main loop
+    static constexpr int MIN_BLOCKS = (ATM && !GATEUP) ? 2 : 1;
+    static constexpr int STAGES = 4;
+    static constexpr int A_SMEM = ATM ? 0 : (GATEUP ? 2 : 1) * A_TILE;  // A bytes per shared-memory stage
+    static constexpr int STAGE = A_SMEM + B_TILE;
+    static constexpr int ACC_COLS = GATEUP ? 256 : 128;                  // fp32 accumulators
+    static constexpr int A_COLS = ATM ? (GATEUP ? 2 : 1) * (BK / 2) : 0;  // TMEM columns of one stage's A tiles
+    static constexpr int TMEM_COLS = ATM ? (GATEUP ? 512 : 256) : ACC_COLS;
+    static_assert(ACC_COLS + STAGES * A_COLS <= TMEM_COLS, "tensor memory");
     static constexpr int PRING_OFF = STAGES * STAGE;
     static constexpr int TABLE_OFF = PRING_OFF + PackTma<AFMT, GATEUP>::NSLOT * PackTma<AFMT, GATEUP>::SLOT;
-    static constexpr int SMEM = TABLE_OFF + TABLE_BYTES + 1024;  // + alignment slack
+    static constexpr int TBL = AFMT == DS4MOE_FMT_IQ2X ? TABLE_BYTES : 0;  // only IQ2X dequantizes via a table
+    static constexpr int SMEM = TABLE_OFF + TBL + 1024;  // + alignment slack
     static_assert(SMEM <= 232448, "shared memory");
 };
 
@@ -153,6 +174,34 @@ __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t adesc, uint64_
         "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\ttcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(
             d_tmem),
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+// Same MMA with A read from tensor memory (a_tmem: lane 0, first column of a 128 x 16 fp16 tile).
+__device__ __forceinline__ void mma_f16_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                           uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\ttcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(
+            d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+// 32 consecutive 32-bit columns of this thread's TMEM lane (warp-collective), then wait for the stores.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,"
+        "%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};\n\t"
+        "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+        "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]),
+        "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
+        "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};\n\t"
+        "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+        "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
 }
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
@@ -361,7 +410,7 @@ __device__ __forceinline__ void sp_dequant(const SPack<AFMT, GATEUP> &pk, int h,
 // ---- the kernel -------------------------------------------------------------------------------------------
 
 template <int AFMT, bool GATEUP>
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __launch_bounds__(THREADS, Cfg<AFMT, GATEUP>::MIN_BLOCKS)
     grouped_tc_kernel(GroupedArgs a, const __grid_constant__ CUtensorMap tmap_b, const __grid_constant__ CUtensorMap tmap_a0,
                       const __grid_constant__ CUtensorMap tmap_a1, const __grid_constant__ CUtensorMap pmap0,
                       const __grid_constant__ CUtensorMap pmap1, const __grid_constant__ CUtensorMap pmap2,
@@ -464,12 +513,18 @@ __global__ void __launch_bounds__(THREADS, 1)
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t st = smem_u32(smem + s * C::STAGE);
-                const uint32_t a0 = st, a1 = st + A_TILE, b0 = st + (GATEUP ? 2 : 1) * A_TILE;
+                const uint32_t a0 = st, a1 = st + A_TILE, b0 = st + C::A_SMEM;
+                const uint32_t at0 = tmem + C::ACC_COLS + s * C::A_COLS;  // ATM: gate A columns, up at +BK/2
 #pragma unroll
                 for (int kk = 0; kk < BK / 16; kk++) {
                     const uint32_t acc = (kc > 0 || kk > 0) ? 1u : 0u;
-                    mma_f16(tmem, smem_desc(a0 + kk * 32), smem_desc(b0 + kk * 32), idesc, acc);
-                    if constexpr (GATEUP) mma_f16(tmem + NT, smem_desc(a1 + kk * 32), smem_desc(b0 + kk * 32), idesc, acc);
+                    if constexpr (C::ATM) {
+                        mma_f16_ta(tmem, at0 + kk * 8, smem_desc(b0 + kk * 32), idesc, acc);
+                        if constexpr (GATEUP) mma_f16_ta(tmem + NT, at0 + BK / 2 + kk * 8, smem_desc(b0 + kk * 32), idesc, acc);
+                    } else {
+                        mma_f16(tmem, smem_desc(a0 + kk * 32), smem_desc(b0 + kk * 32), idesc, acc);
+                        if constexpr (GATEUP) mma_f16(tmem + NT, smem_desc(a1 + kk * 32), smem_desc(b0 + kk * 32), idesc, acc);
+                    }
                 }
                 mma_commit(empty(s));
             }
@@ -484,7 +539,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const int s = kc % S;
                 const uint32_t par = ((kc / S) & 1) ^ 1;
                 if (!mbar_wait(empty(s), par, abort_flag)) break;
-                const uint32_t st = smem_u32(smem + s * C::STAGE), bst = st + (GATEUP ? 2 : 1) * A_TILE;
+                const uint32_t st = smem_u32(smem + s * C::STAGE), bst = st + C::A_SMEM;
                 // full boxes: rows past a tensor's end are zero-filled and still counted
                 mbar_expect_tx(full_b(s), B_TILE + (DENSE ? (GATEUP ? 2 : 1) * A_TILE : 0));
                 if constexpr (DENSE) {
@@ -534,12 +589,42 @@ __global__ void __launch_bounds__(THREADS, 1)
         __syncwarp();
     } else {
         // ------------------------------------------------------------------ dequantizing producers
+        // Hands this thread's dequantized part of stage s (row R of matrix m, or K half h of a DOWN row) to the
+        // MMA, then arrives on the stage's barrier.  A in TMEM: row R is TMEM lane R (a warp may store only to
+        // its lane quarter, warp & 3), fp16 K pairs in 32-bit columns.  A in shared memory: the 128-byte-swizzled
+        // K-major tile the MMA descriptor describes.  Either way the writing thread makes its own stores visible
+        // to the tensor core (async proxy) and releases them itself.
+        auto put_a = [&](int s, int m, int R, int h, const auto &o) {
+            constexpr int NOUT = GATEUP ? 8 : 4;
+            if constexpr (C::ATM) {
+                uint32_t wv[NOUT * 4];
+#pragma unroll
+                for (int c = 0; c < NOUT; c++) {
+                    wv[4 * c] = o[c].x; wv[4 * c + 1] = o[c].y; wv[4 * c + 2] = o[c].z; wv[4 * c + 3] = o[c].w;
+                }
+                __syncwarp();
+                tc_fence_after();  // after the stage-release wait: the MMA that read these columns is done
+                const uint32_t ta = tmem + (uint32_t((warp & 3) * 32) << 16) + C::ACC_COLS + s * C::A_COLS;
+                if constexpr (GATEUP) tmem_st32(ta + m * (BK / 2), wv);
+                else tmem_st16(ta + h * (BK / 4), wv);
+                tc_fence_before();
+            } else {
+                uint8_t *ast = smem + s * C::STAGE + m * A_TILE;
+#pragma unroll
+                for (int c = 0; c < NOUT; c++)
+                    *reinterpret_cast<uint4 *>(ast + swz(R, (GATEUP ? 0 : h * 4) + c)) = o[c];
+                fence_proxy_async();
+            }
+            mbar_arrive(full_a(s));
+        };
         if constexpr (PT::ON) {
             constexpr int NOUT = GATEUP ? 8 : 4;
             const int at = tid - W_A0 * 32;  // 0 .. 255
             const int m = GATEUP ? at >> 7 : 0;
-            const int R = GATEUP ? at & 127 : at >> 1;
-            const int h = GATEUP ? 0 : at & 1;
+            // DOWN with A in TMEM: a warp may store only to its TMEM lane quarter (warp & 3), so warps 4-7 take
+            // the first K half of rows 32q..32q+31 and warps 8-11 the second
+            const int R = GATEUP ? at & 127 : (C::ATM ? (warp & 3) * 32 + lane : at >> 1);
+            const int h = GATEUP ? 0 : (C::ATM ? (warp - W_A0) >> 2 : at & 1);
             const uint8_t *mat = GATEUP && m ? a.a1 + size_t(e) * a.a1_stride : a.a0 + size_t(e) * a.a_stride;
             const size_t rowb = size_t(blockIdx.x * M + R) * nss_p;  // block index of the row's first block
             const uint8_t *tbl_lane = tbl + (lane & 7) * 16;
@@ -605,14 +690,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                     else if (jj == 1) sp_dequant<AFMT, GATEUP, 1>(cur, h, ss, tbl_lane, o, inf, hsc);
                     else if (jj == 2) sp_dequant<AFMT, GATEUP, 2>(cur, h, ss, tbl_lane, o, inf, hsc);
                     else sp_dequant<AFMT, GATEUP, 3>(cur, h, ss, tbl_lane, o, inf, hsc);
-                    uint8_t *ast = smem + s * C::STAGE + m * A_TILE;
-#pragma unroll
-                    for (int c = 0; c < NOUT; c++)
-                        *reinterpret_cast<uint4 *>(ast + swz(R, (GATEUP ? 0 : h * 4) + c)) = o[c];
-                    // each writing thread makes its own stores visible to the tensor core (async proxy) and
-                    // releases them itself
-                    fence_proxy_async();
-                    mbar_arrive(full_a(s));
+                    put_a(s, m, R, h, o);
                 }
             }
             if (inf) set_device_error(DS4MOE_EDEVICE);
@@ -621,14 +699,15 @@ __global__ void __launch_bounds__(THREADS, 1)
             constexpr int NOUT = GATEUP ? 8 : 4;
             const int at = tid - W_A0 * 32;  // 0 .. 255
             const int m = GATEUP ? at >> 7 : 0;
-            const int R = GATEUP ? at & 127 : at >> 1;
-            const int h = GATEUP ? 0 : at & 1;
+            const int R = GATEUP ? at & 127 : (C::ATM ? (warp & 3) * 32 + lane : at >> 1);  // as in the path above
+            const int h = GATEUP ? 0 : (C::ATM ? (warp - W_A0) >> 2 : at & 1);
             const uint8_t *mat = GATEUP && m ? a.a1 + size_t(e) * a.a1_stride : a.a0 + size_t(e) * a.a_stride;
             const int row = blockIdx.x * M + R;
             const uint8_t *tbl_lane = tbl + (lane & 7) * 16;
             const int nss = nk / SS;
             // packed data of PF super-stages is in flight: super-stage ss+PF-1 is requested while ss is consumed
-            constexpr int PF = SPackCfg<AFMT, GATEUP>::NW <= 20 ? 3 : 2;
+            // (two when two CTAs share the SM: their warps hide the latency, and the registers are halved)
+            constexpr int PF = SPackCfg<AFMT, GATEUP>::NW <= 20 && C::MIN_BLOCKS == 1 ? 3 : 2;
             SPack<AFMT, GATEUP> pf[PF];
     #pragma unroll
             for (int p = 0; p < PF - 1; p++)
@@ -664,12 +743,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                         } else {
                             sp_dequant<AFMT, GATEUP, 0>(cur, h, ss, tbl_lane, o, inf);
                         }
-                        uint8_t *ast = smem + s * C::STAGE + m * A_TILE;
-    #pragma unroll
-                        for (int c = 0; c < NOUT; c++)
-                            *reinterpret_cast<uint4 *>(ast + swz(R, (GATEUP ? 0 : h * 4) + c)) = o[c];
-                        fence_proxy_async();
-                        mbar_arrive(full_a(s));
+                        put_a(s, m, R, h, o);
                     }
                 }
             }
