@@ -17,16 +17,13 @@
 //               256-wide K block at a time, with 3D TMA copies into a 2-slot
 //               shared-memory ring (Q4K and bf16 producers load into registers).
 //   warps 4-11  dequantize the packed blocks in registers (shared-memory
-//               codebook / sign-bit XOR / fp16 scale) and hand the fp16 A
-//               tiles to the MMA: for the IQ2X gate/up and the packed down
-//               kernels they go to tensor memory (tcgen05.st, row = TMEM
-//               lane) and the MMA reads A from there, which keeps them out of
-//               shared memory (the MMA's operand reads and the producers'
-//               stores share its bandwidth); the Q4K gate/up kernel writes
-//               them to shared memory in the swizzled K-major layout the MMA
-//               descriptor describes.  Warps 4-7 then run the epilogue:
-//               tcgen05.ld the accumulators, SwiGLU (gate/up) or
-//               routing-weight scaling (down), stores.
+//               codebook / sign-bit XOR / fp16 scale) and store the fp16 A
+//               tiles to tensor memory (tcgen05.st, row = TMEM lane); the MMA
+//               reads A from there, which keeps the A tiles out of shared
+//               memory (the MMA's operand reads, the producers' stores and the
+//               codebook lookups would otherwise share its bandwidth).  Warps
+//               4-7 then run the epilogue: tcgen05.ld the accumulators, SwiGLU
+//               (gate/up) or routing-weight scaling (down), stores.
 //
 // The packed down kernels need 256 TMEM columns and ~90 KB of shared memory,
 // so two CTAs share an SM and one's prologue and epilogue overlap the other's
@@ -79,8 +76,9 @@ struct PackTma {
 template <int AFMT, bool GATEUP>
 struct Cfg {
     // ATM: the dequantized A tiles live in tensor memory (tcgen05.st by the producers, MMA with A from TMEM);
-    // the shared-memory stages then hold only the token tile
-    static constexpr bool ATM = (AFMT == DS4MOE_FMT_IQ2X && GATEUP) || (!is_dense<AFMT>() && !GATEUP);
+    // the shared-memory stages then hold only the token tile.  Every packed format does this; dense A tiles
+    // come by TMA into shared memory.
+    static constexpr bool ATM = !is_dense<AFMT>();
     // the packed down kernels then fit twice per SM (shared memory, TMEM, registers), so one CTA's prologue and
     // epilogue overlap the other's main loop
     static constexpr int MIN_BLOCKS = (ATM && !GATEUP) ? 2 : 1;
@@ -590,31 +588,22 @@ __global__ void __launch_bounds__(THREADS, Cfg<AFMT, GATEUP>::MIN_BLOCKS)
     } else {
         // ------------------------------------------------------------------ dequantizing producers
         // Hands this thread's dequantized part of stage s (row R of matrix m, or K half h of a DOWN row) to the
-        // MMA, then arrives on the stage's barrier.  A in TMEM: row R is TMEM lane R (a warp may store only to
-        // its lane quarter, warp & 3), fp16 K pairs in 32-bit columns.  A in shared memory: the 128-byte-swizzled
-        // K-major tile the MMA descriptor describes.  Either way the writing thread makes its own stores visible
-        // to the tensor core (async proxy) and releases them itself.
-        auto put_a = [&](int s, int m, int R, int h, const auto &o) {
+        // MMA through tensor memory, then arrives on the stage's barrier: row R is TMEM lane R (a warp may store
+        // only to its lane quarter, warp & 3), fp16 K pairs in 32-bit columns.  The writing thread waits for its
+        // own stores (tcgen05.wait::st) and releases them itself.
+        auto put_a = [&](int s, int m, int h, const auto &o) {
             constexpr int NOUT = GATEUP ? 8 : 4;
-            if constexpr (C::ATM) {
-                uint32_t wv[NOUT * 4];
+            uint32_t wv[NOUT * 4];
 #pragma unroll
-                for (int c = 0; c < NOUT; c++) {
-                    wv[4 * c] = o[c].x; wv[4 * c + 1] = o[c].y; wv[4 * c + 2] = o[c].z; wv[4 * c + 3] = o[c].w;
-                }
-                __syncwarp();
-                tc_fence_after();  // after the stage-release wait: the MMA that read these columns is done
-                const uint32_t ta = tmem + (uint32_t((warp & 3) * 32) << 16) + C::ACC_COLS + s * C::A_COLS;
-                if constexpr (GATEUP) tmem_st32(ta + m * (BK / 2), wv);
-                else tmem_st16(ta + h * (BK / 4), wv);
-                tc_fence_before();
-            } else {
-                uint8_t *ast = smem + s * C::STAGE + m * A_TILE;
-#pragma unroll
-                for (int c = 0; c < NOUT; c++)
-                    *reinterpret_cast<uint4 *>(ast + swz(R, (GATEUP ? 0 : h * 4) + c)) = o[c];
-                fence_proxy_async();
+            for (int c = 0; c < NOUT; c++) {
+                wv[4 * c] = o[c].x; wv[4 * c + 1] = o[c].y; wv[4 * c + 2] = o[c].z; wv[4 * c + 3] = o[c].w;
             }
+            __syncwarp();
+            tc_fence_after();  // after the stage-release wait: the MMA that read these columns is done
+            const uint32_t ta = tmem + (uint32_t((warp & 3) * 32) << 16) + C::ACC_COLS + s * C::A_COLS;
+            if constexpr (GATEUP) tmem_st32(ta + m * (BK / 2), wv);
+            else tmem_st16(ta + h * (BK / 4), wv);
+            tc_fence_before();
             mbar_arrive(full_a(s));
         };
         if constexpr (PT::ON) {
@@ -690,7 +679,7 @@ __global__ void __launch_bounds__(THREADS, Cfg<AFMT, GATEUP>::MIN_BLOCKS)
                     else if (jj == 1) sp_dequant<AFMT, GATEUP, 1>(cur, h, ss, tbl_lane, o, inf, hsc);
                     else if (jj == 2) sp_dequant<AFMT, GATEUP, 2>(cur, h, ss, tbl_lane, o, inf, hsc);
                     else sp_dequant<AFMT, GATEUP, 3>(cur, h, ss, tbl_lane, o, inf, hsc);
-                    put_a(s, m, R, h, o);
+                    put_a(s, m, h, o);
                 }
             }
             if (inf) set_device_error(DS4MOE_EDEVICE);
@@ -743,7 +732,7 @@ __global__ void __launch_bounds__(THREADS, Cfg<AFMT, GATEUP>::MIN_BLOCKS)
                         } else {
                             sp_dequant<AFMT, GATEUP, 0>(cur, h, ss, tbl_lane, o, inf);
                         }
-                        put_a(s, m, R, h, o);
+                        put_a(s, m, h, o);
                     }
                 }
             }
