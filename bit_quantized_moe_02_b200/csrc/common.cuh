@@ -89,7 +89,10 @@ __device__ __forceinline__ int pow2_exponent_for(float amax, int top) {
     return max(-100, min(100, e));
 }
 
-__device__ __forceinline__ float silu(float g) { return g / (1.f + expf(-g)); }
+// silu(g) = g * sigmoid(g), with the fast hardware exponential and divide (relative error ~1e-6, far inside the
+// layer's tolerance).  For g below about -88 the denominator overflows to +inf and the result is -0; the exact
+// value is smaller than 1e-36 in magnitude.
+__device__ __forceinline__ float silu(float g) { return __fdividef(g, 1.f + __expf(-g)); }
 
 // Programmatic dependent launch: wait for the preceding grid's results.
 // A no-op when the kernel was launched without the PDL attribute.

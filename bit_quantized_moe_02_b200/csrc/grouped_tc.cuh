@@ -21,9 +21,10 @@
 //               tiles to tensor memory (tcgen05.st, row = TMEM lane); the MMA
 //               reads A from there, which keeps the A tiles out of shared
 //               memory (the MMA's operand reads, the producers' stores and the
-//               codebook lookups would otherwise share its bandwidth).  Warps
-//               4-7 then run the epilogue: tcgen05.ld the accumulators, SwiGLU
-//               (gate/up) or routing-weight scaling (down), stores.
+//               codebook lookups would otherwise share its bandwidth).  All
+//               eight then run the epilogue, splitting the token columns:
+//               tcgen05.ld the accumulators, SwiGLU (gate/up) or
+//               routing-weight scaling (down), stores.
 //
 // The packed down kernels need 256 TMEM columns and ~90 KB of shared memory,
 // so two CTAs share an SM and one's prologue and epilogue overlap the other's
@@ -739,10 +740,13 @@ __global__ void __launch_bounds__(THREADS, Cfg<AFMT, GATEUP>::MIN_BLOCKS)
             if (inf) set_device_error(DS4MOE_EDEVICE);
         }
 
-        // ------------------------------------------------------------------ epilogue (warps 4..7)
-        if (warp < W_A0 + 4) {
-            const int q = warp - W_A0;  // TMEM lane quarter
+        // ------------------------------------------------------------------ epilogue (warps 4..11)
+        // Warps 4-7 and 8-11 cover the same TMEM lane quarters (warp & 3); they split the tile's token columns
+        // in 32-wide chunks, so that two warps per scheduler hide each other's latencies.
+        {
+            const int q = warp & 3;  // TMEM lane quarter
             const int r = q * 32 + lane;
+            const int c_first = ((warp - W_A0) >> 2) * 32;
             const bool ok = __all_sync(0xffffffffu, mbar_wait(accum_bar, 0, abort_flag) && !*abort_flag);
             tc_fence_after();
             const uint32_t tq = tmem + (uint32_t(q * 32) << 16);
@@ -753,7 +757,7 @@ __global__ void __launch_bounds__(THREADS, Cfg<AFMT, GATEUP>::MIN_BLOCKS)
                 // needs no scale).  The down GEMM multiplies this K range of its weights by 2^e.
                 constexpr bool F16OUT = AFMT != FMT_BF16D;
                 auto store_pass = [&](float osc, uint32_t &amax_bits) {
-                    for (int c0 = 0; c0 < n_eff; c0 += 32) {
+                    for (int c0 = c_first; c0 < n_eff; c0 += 64) {
                         uint32_t g[32], u[32];
                         tmem_ld32(tq + c0, g);
                         tmem_ld32(tq + NT + c0, u);
@@ -776,7 +780,7 @@ __global__ void __launch_bounds__(THREADS, Cfg<AFMT, GATEUP>::MIN_BLOCKS)
                 if (ok) store_pass(1.f, amax_bits);
                 amax_bits = __reduce_max_sync(0xffffffffu, amax_bits);
                 if (lane == 0) atomicMax(&s_hmax, amax_bits);
-                asm volatile("bar.sync 1, 128;" ::: "memory");  // the four epilogue warps
+                asm volatile("bar.sync 1, 256;" ::: "memory");  // the eight epilogue warps
                 const uint32_t tmax = *reinterpret_cast<volatile uint32_t *>(&s_hmax);
                 int he = 0;
                 if (tmax >= 0x7F800000u) {
@@ -788,11 +792,11 @@ __global__ void __launch_bounds__(THREADS, Cfg<AFMT, GATEUP>::MIN_BLOCKS)
                     uint32_t unused = 0;
                     if (ok) store_pass(ldexpf(1.f, -he), unused);
                 }
-                if (ok && r == 0 && a.h_exp_out) a.h_exp_out[int(blockIdx.y) * gridDim.x + blockIdx.x] = he;
+                if (ok && r == 0 && c_first == 0 && a.h_exp_out) a.h_exp_out[int(blockIdx.y) * gridDim.x + blockIdx.x] = he;
             } else {
                 if (ok) {
                     float *out = reinterpret_cast<float *>(a.out);
-                    for (int c0 = 0; c0 < n_eff; c0 += 32) {
+                    for (int c0 = c_first; c0 < n_eff; c0 += 64) {
                         uint32_t g[32];
                         tmem_ld32(tq + c0, g);
                         if (a.out_row) {
