@@ -122,7 +122,10 @@ constexpr int DG_THREADS = DG_WARPS * 32;
 constexpr uint32_t DG_TABLE_ABS = 0x10000;  // absolute shared address of the 64 KB codebook table
 constexpr int DG_ROWS = 4;                  // gate/up row pairs per unit (routed and shared): 4 or 8
 constexpr int DG_MAX_D = 8192;
-constexpr int DG_RING = 4;                  // row slices whose packed data is in flight per lane (divides 2 DG_ROWS)
+// Row slices whose packed data is in flight per lane (divides 2 DG_ROWS): all eight row-matrices of a unit for
+// IQ2X (its slices are 22 bytes a lane); four for Q4K, whose larger slices would otherwise spill at 128 registers.
+template <int FMT>
+__host__ __device__ constexpr int dg_ring() { return FMT == DS4MOE_FMT_Q4K ? 4 : 8; }
 
 // Contraction lengths the gate/up kernel takes: d = 256 * nblk with nblk in {1, 2, 4, 8, 16, 32}.  A lane owns
 // VPP = min(nblk, 8) consecutive 8-vectors of a row per pass; nblk / VPP passes.
@@ -441,9 +444,10 @@ __global__ void __launch_bounds__(DG_THREADS, 1)
             else
                 iq_rp_load<VPP>(R, rr & 1 ? U : G, ex.pg, r0 + (rr >> 1), nblk, (t / NRR) * 32 * VPP + lane * VPP);
         };
-        Rp ring[DG_RING];
+        constexpr int RING = dg_ring<FMT>();
+        Rp ring[RING];
 #pragma unroll
-        for (int s = 0; s < DG_RING; s++) load(ring[s], s);
+        for (int s = 0; s < RING; s++) load(ring[s], s);
         for (int p = 0; p < npass; p++) {
             const int v0 = p * 32 * VPP + lane * VPP;
             uint4 xr[VPP];
@@ -456,10 +460,10 @@ __global__ void __launch_bounds__(DG_THREADS, 1)
             }
 #pragma unroll
             for (int rr = 0; rr < NRR; rr++) {
-                if constexpr (Q4) acc[rr] += q4_rp_dot<VPP>(ring[rr % DG_RING], xr, xsv, v0, lane_tbl);
-                else acc[rr] += iq_rp_dot<VPP>(ring[rr % DG_RING], xr, v0, lane_tbl);
-                const int tn = p * NRR + rr + DG_RING;
-                if (tn < T) load(ring[rr % DG_RING], tn);
+                if constexpr (Q4) acc[rr] += q4_rp_dot<VPP>(ring[rr % RING], xr, xsv, v0, lane_tbl);
+                else acc[rr] += iq_rp_dot<VPP>(ring[rr % RING], xr, v0, lane_tbl);
+                const int tn = p * NRR + rr + RING;
+                if (tn < T) load(ring[rr % RING], tn);
             }
         }
         const float v = reduce_scatter<NRR>(acc, lane);
