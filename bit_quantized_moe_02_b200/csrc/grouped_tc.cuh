@@ -421,7 +421,7 @@ __global__ void __launch_bounds__(THREADS, Cfg<AFMT, GATEUP>::MIN_BLOCKS)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *tbl = smem + C::TABLE_OFF;
-    __shared__ __align__(8) uint64_t bars[3 * 4 + 1 + 4];  // full_a[S], full_b[S], empty[S], accum, packed ring
+    __shared__ __align__(8) uint64_t bars[3 * 4 + 1 + 4];  // (unused)[S], full[S], empty[S], accum, packed ring
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
     __shared__ float s_colsc[NT];
@@ -445,8 +445,10 @@ __global__ void __launch_bounds__(THREADS, Cfg<AFMT, GATEUP>::MIN_BLOCKS)
     const int n_eff = max(16, (cnt + 15) & ~15);
     const int nk = a.K / BK;
 
-    auto full_a = [&](int s) { return smem_u32(&bars[s]); };
+    // One "stage full" barrier per stage: the token-tile TMA (its expect-tx arrival and bytes) and, for packed
+    // formats, every producer thread (its A part) arrive on it, so the MMA issuer waits once per stage.
     auto full_b = [&](int s) { return smem_u32(&bars[4 + s]); };
+    auto full_a = full_b;
     auto empty = [&](int s) { return smem_u32(&bars[8 + s]); };
     const uint32_t accum_bar = smem_u32(&bars[12]);
     auto full_p = [&](int s) { return smem_u32(&bars[13 + s]); };
@@ -455,8 +457,7 @@ __global__ void __launch_bounds__(THREADS, Cfg<AFMT, GATEUP>::MIN_BLOCKS)
 
     if (tid == 0) {
         for (int s = 0; s < S; s++) {
-            mbar_init(full_a(s), N_WA * 32);  // every producer thread arrives (see the producers)
-            mbar_init(full_b(s), 1);
+            mbar_init(full_b(s), DENSE ? 1 : N_WA * 32 + 1);  // TMA arrival + every producer thread
             mbar_init(empty(s), 1);
         }
         mbar_init(accum_bar, 1);
@@ -508,7 +509,7 @@ __global__ void __launch_bounds__(THREADS, Cfg<AFMT, GATEUP>::MIN_BLOCKS)
             for (int kc = 0; kc < nk && ok; kc++) {
                 const int s = kc % S;
                 const uint32_t par = (kc / S) & 1;
-                ok = (DENSE || mbar_wait(full_a(s), par, abort_flag)) && mbar_wait(full_b(s), par, abort_flag);
+                ok = mbar_wait(full_b(s), par, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t st = smem_u32(smem + s * C::STAGE);
@@ -549,7 +550,8 @@ __global__ void __launch_bounds__(THREADS, Cfg<AFMT, GATEUP>::MIN_BLOCKS)
                 issued = kc + 1;
             }
             if (*abort_flag) {
-                // let this CTA's copies still in flight land before its shared memory is released (bounded)
+                // let this CTA's copies still in flight land before its shared memory is released (bounded: the
+                // stage barrier also counts the producers, so after an abort this may run to its time limit)
                 const uint64_t t0 = globaltimer();
                 for (int kc = max(0, issued - S); kc < issued; kc++)
                     while (!mbar_try_wait(full_b(kc % S), (kc / S) & 1) && globaltimer() - t0 < uint64_t(WAIT_NS)) {
