@@ -83,11 +83,15 @@ struct Cfg {
     // the packed down kernels then fit twice per SM (shared memory, TMEM, registers), so one CTA's prologue and
     // epilogue overlap the other's main loop
     static constexpr int MIN_BLOCKS = (ATM && !GATEUP) ? 2 : 1;
-    static constexpr int STAGES = 4;
+    // K per pipeline step: 128 for the packed kernels (two 64-wide sub-steps: two token-tile boxes, two A parts
+    // per producer), which halves the per-step barrier, fence and commit work; 64 for the dense ones
+    static constexpr int KS = ATM ? 2 * BK : BK;
+    static constexpr int SUB = KS / BK;
+    static constexpr int STAGES = ATM ? 2 : 4;
     static constexpr int A_SMEM = ATM ? 0 : (GATEUP ? 2 : 1) * A_TILE;  // A bytes per shared-memory stage
-    static constexpr int STAGE = A_SMEM + B_TILE;
+    static constexpr int STAGE = A_SMEM + SUB * B_TILE;
     static constexpr int ACC_COLS = GATEUP ? 256 : 128;                  // fp32 accumulators
-    static constexpr int A_COLS = ATM ? (GATEUP ? 2 : 1) * (BK / 2) : 0;  // TMEM columns of one stage's A tiles
+    static constexpr int A_COLS = ATM ? (GATEUP ? 2 : 1) * (KS / 2) : 0;  // TMEM columns of one stage's A tiles
     static constexpr int TMEM_COLS = ATM ? (GATEUP ? 512 : 256) : ACC_COLS;
     static_assert(ACC_COLS + STAGES * A_COLS <= TMEM_COLS, "tensor memory");
     static constexpr int PRING_OFF = STAGES * STAGE;
@@ -443,7 +447,7 @@ __global__ void __launch_bounds__(THREADS, Cfg<AFMT, GATEUP>::MIN_BLOCKS)
         cnt = min(NT, a.n_pos - pos0);
     }
     const int n_eff = max(16, (cnt + 15) & ~15);
-    const int nk = a.K / BK;
+    const int nk = a.K / C::KS;  // pipeline steps
 
     // One "stage full" barrier per stage: the token-tile TMA (its expect-tx arrival and bytes) and, for packed
     // formats, every producer thread (its A part) arrive on it, so the MMA issuer waits once per stage.
@@ -514,13 +518,14 @@ __global__ void __launch_bounds__(THREADS, Cfg<AFMT, GATEUP>::MIN_BLOCKS)
                 tc_fence_after();
                 const uint32_t st = smem_u32(smem + s * C::STAGE);
                 const uint32_t a0 = st, a1 = st + A_TILE, b0 = st + C::A_SMEM;
-                const uint32_t at0 = tmem + C::ACC_COLS + s * C::A_COLS;  // ATM: gate A columns, up at +BK/2
+                const uint32_t at0 = tmem + C::ACC_COLS + s * C::A_COLS;  // ATM: gate A columns, up at +KS/2
 #pragma unroll
-                for (int kk = 0; kk < BK / 16; kk++) {
+                for (int kk = 0; kk < C::KS / 16; kk++) {
                     const uint32_t acc = (kc > 0 || kk > 0) ? 1u : 0u;
                     if constexpr (C::ATM) {
-                        mma_f16_ta(tmem, at0 + kk * 8, smem_desc(b0 + kk * 32), idesc, acc);
-                        if constexpr (GATEUP) mma_f16_ta(tmem + NT, at0 + BK / 2 + kk * 8, smem_desc(b0 + kk * 32), idesc, acc);
+                        const uint64_t bd = smem_desc(b0 + (kk / 4) * B_TILE + (kk % 4) * 32);  // 64-wide sub-tile, 16-wide slice
+                        mma_f16_ta(tmem, at0 + kk * 8, bd, idesc, acc);
+                        if constexpr (GATEUP) mma_f16_ta(tmem + NT, at0 + C::KS / 2 + kk * 8, bd, idesc, acc);
                     } else {
                         mma_f16(tmem, smem_desc(a0 + kk * 32), smem_desc(b0 + kk * 32), idesc, acc);
                         if constexpr (GATEUP) mma_f16(tmem + NT, smem_desc(a1 + kk * 32), smem_desc(b0 + kk * 32), idesc, acc);
@@ -541,12 +546,14 @@ __global__ void __launch_bounds__(THREADS, Cfg<AFMT, GATEUP>::MIN_BLOCKS)
                 if (!mbar_wait(empty(s), par, abort_flag)) break;
                 const uint32_t st = smem_u32(smem + s * C::STAGE), bst = st + C::A_SMEM;
                 // full boxes: rows past a tensor's end are zero-filled and still counted
-                mbar_expect_tx(full_b(s), B_TILE + (DENSE ? (GATEUP ? 2 : 1) * A_TILE : 0));
+                mbar_expect_tx(full_b(s), C::SUB * B_TILE + (DENSE ? (GATEUP ? 2 : 1) * A_TILE : 0));
                 if constexpr (DENSE) {
                     tma_load_2d(st, &tmap_a0, kc * BK, blockIdx.x * M, full_b(s));
                     if constexpr (GATEUP) tma_load_2d(st + A_TILE, &tmap_a1, kc * BK, blockIdx.x * M, full_b(s));
                 }
-                tma_load_2d(bst, &tmap_b, kc * BK, pos0, full_b(s));
+#pragma unroll
+                for (int sub = 0; sub < C::SUB; sub++)
+                    tma_load_2d(bst + sub * B_TILE, &tmap_b, kc * C::KS + sub * BK, pos0, full_b(s));
                 issued = kc + 1;
             }
             if (*abort_flag) {
@@ -594,18 +601,24 @@ __global__ void __launch_bounds__(THREADS, Cfg<AFMT, GATEUP>::MIN_BLOCKS)
         // MMA through tensor memory, then arrives on the stage's barrier: row R is TMEM lane R (a warp may store
         // only to its lane quarter, warp & 3), fp16 K pairs in 32-bit columns.  The writing thread waits for its
         // own stores (tcgen05.wait::st) and releases them itself.
-        auto put_a = [&](int s, int m, int h, const auto &o) {
+        // A step's A tile is C::KS / 2 columns per matrix; 64-wide sub-step js takes columns [32 js, 32 js + 32),
+        // of which a DOWN thread's K half h writes [32 js + 16 h, 32 js + 16 h + 16).
+        auto begin_a = [&]() {
+            __syncwarp();
+            tc_fence_after();  // after the stage-release wait: the MMA that read these columns is done
+        };
+        auto st_a = [&](int s, int m, int h, int js, const auto &o) {
             constexpr int NOUT = GATEUP ? 8 : 4;
             uint32_t wv[NOUT * 4];
 #pragma unroll
             for (int c = 0; c < NOUT; c++) {
                 wv[4 * c] = o[c].x; wv[4 * c + 1] = o[c].y; wv[4 * c + 2] = o[c].z; wv[4 * c + 3] = o[c].w;
             }
-            __syncwarp();
-            tc_fence_after();  // after the stage-release wait: the MMA that read these columns is done
-            const uint32_t ta = tmem + (uint32_t((warp & 3) * 32) << 16) + C::ACC_COLS + s * C::A_COLS;
-            if constexpr (GATEUP) tmem_st32(ta + m * (BK / 2), wv);
+            const uint32_t ta = tmem + (uint32_t((warp & 3) * 32) << 16) + C::ACC_COLS + s * C::A_COLS + js * (BK / 2);
+            if constexpr (GATEUP) tmem_st32(ta + m * (C::KS / 2), wv);
             else tmem_st16(ta + h * (BK / 4), wv);
+        };
+        auto end_a = [&](int s) {
             tc_fence_before();
             mbar_arrive(full_a(s));
         };
@@ -667,22 +680,29 @@ __global__ void __launch_bounds__(THREADS, Cfg<AFMT, GATEUP>::MIN_BLOCKS)
                 fence_proxy_async();
                 mbar_arrive(empty_p(sl));
                 s00 = s10; s01 = s11; s10 = s20; s11 = s21;
+                constexpr int SPB = 4 / C::SUB;  // pipeline steps per 256-wide block
 #pragma unroll
-                for (int jj = 0; jj < 4; jj++) {
-                    const int kc = ss * 4 + jj;
+                for (int jj = 0; jj < SPB; jj++) {
+                    const int kc = ss * SPB + jj;
                     const int s = kc % S;
                     const uint32_t par = ((kc / S) & 1) ^ 1;
                     if (!mbar_wait(empty(s), par, abort_flag)) {
                         run = false;
                         break;
                     }
-                    uint4 o[NOUT];
-                    const float hsc = GATEUP ? 1.f : s_hsc[kc >> 1];
-                    if (jj == 0) sp_dequant<AFMT, GATEUP, 0>(cur, h, ss, tbl_lane, o, inf, hsc);
-                    else if (jj == 1) sp_dequant<AFMT, GATEUP, 1>(cur, h, ss, tbl_lane, o, inf, hsc);
-                    else if (jj == 2) sp_dequant<AFMT, GATEUP, 2>(cur, h, ss, tbl_lane, o, inf, hsc);
-                    else sp_dequant<AFMT, GATEUP, 3>(cur, h, ss, tbl_lane, o, inf, hsc);
-                    put_a(s, m, h, o);
+                    begin_a();
+#pragma unroll
+                    for (int js = 0; js < C::SUB; js++) {
+                        const int J = jj * C::SUB + js;  // 64-wide stage of the block
+                        uint4 o[NOUT];
+                        const float hsc = GATEUP ? 1.f : s_hsc[(kc * C::KS + js * BK) >> 7];
+                        if (J == 0) sp_dequant<AFMT, GATEUP, 0>(cur, h, ss, tbl_lane, o, inf, hsc);
+                        else if (J == 1) sp_dequant<AFMT, GATEUP, 1>(cur, h, ss, tbl_lane, o, inf, hsc);
+                        else if (J == 2) sp_dequant<AFMT, GATEUP, 2>(cur, h, ss, tbl_lane, o, inf, hsc);
+                        else sp_dequant<AFMT, GATEUP, 3>(cur, h, ss, tbl_lane, o, inf, hsc);
+                        st_a(s, m, h, js, o);
+                    }
+                    end_a(s);
                 }
             }
             if (inf) set_device_error(DS4MOE_EDEVICE);
@@ -696,7 +716,9 @@ __global__ void __launch_bounds__(THREADS, Cfg<AFMT, GATEUP>::MIN_BLOCKS)
             const uint8_t *mat = GATEUP && m ? a.a1 + size_t(e) * a.a1_stride : a.a0 + size_t(e) * a.a_stride;
             const int row = blockIdx.x * M + R;
             const uint8_t *tbl_lane = tbl + (lane & 7) * 16;
-            const int nss = nk / SS;
+            constexpr int SPP = SS / C::SUB;  // pipeline steps per packed super-stage
+            static_assert(SS % C::SUB == 0, "a super-stage holds whole pipeline steps");
+            const int nss = nk / SPP;
             // packed data of PF super-stages is in flight: super-stage ss+PF-1 is requested while ss is consumed
             // (two when two CTAs share the SM: their warps hide the latency, and the registers are halved)
             constexpr int PF = SPackCfg<AFMT, GATEUP>::NW <= 20 && C::MIN_BLOCKS == 1 ? 3 : 2;
@@ -714,28 +736,34 @@ __global__ void __launch_bounds__(THREADS, Cfg<AFMT, GATEUP>::MIN_BLOCKS)
                     if (ss + PF - 1 < nss) sp_load<AFMT, GATEUP>(pf[(q + PF - 1) % PF], mat, a.pa, row, h, a.K, ss + PF - 1);
                     const SPack<AFMT, GATEUP> &cur = pf[q];
     #pragma unroll
-                    for (int jj = 0; jj < SS; jj++) {
-                        const int kc = ss * SS + jj;
+                    for (int jj = 0; jj < SPP; jj++) {
+                        const int kc = ss * SPP + jj;
                         const int s = kc % S;
                         const uint32_t par = ((kc / S) & 1) ^ 1;
                         if (!mbar_wait(empty(s), par, abort_flag)) {
                             run = false;
                             break;
                         }
-                        uint4 o[NOUT];
-                        if constexpr (SS == 4) {
-                            const float hsc = GATEUP ? 1.f : s_hsc[kc >> 1];
-                            if (jj == 0) sp_dequant<AFMT, GATEUP, 0>(cur, h, ss, tbl_lane, o, inf, hsc);
-                            else if (jj == 1) sp_dequant<AFMT, GATEUP, 1>(cur, h, ss, tbl_lane, o, inf, hsc);
-                            else if (jj == 2) sp_dequant<AFMT, GATEUP, 2>(cur, h, ss, tbl_lane, o, inf, hsc);
-                            else sp_dequant<AFMT, GATEUP, 3>(cur, h, ss, tbl_lane, o, inf, hsc);
-                        } else if constexpr (SS == 2) {
-                            if (jj == 0) sp_dequant<AFMT, GATEUP, 0>(cur, h, ss, tbl_lane, o, inf);
-                            else sp_dequant<AFMT, GATEUP, 1>(cur, h, ss, tbl_lane, o, inf);
-                        } else {
-                            sp_dequant<AFMT, GATEUP, 0>(cur, h, ss, tbl_lane, o, inf);
+                        begin_a();
+    #pragma unroll
+                        for (int js = 0; js < C::SUB; js++) {
+                            const int J = jj * C::SUB + js;  // 64-wide stage of the super-stage
+                            uint4 o[NOUT];
+                            if constexpr (SS == 4) {
+                                const float hsc = GATEUP ? 1.f : s_hsc[(kc * C::KS + js * BK) >> 7];
+                                if (J == 0) sp_dequant<AFMT, GATEUP, 0>(cur, h, ss, tbl_lane, o, inf, hsc);
+                                else if (J == 1) sp_dequant<AFMT, GATEUP, 1>(cur, h, ss, tbl_lane, o, inf, hsc);
+                                else if (J == 2) sp_dequant<AFMT, GATEUP, 2>(cur, h, ss, tbl_lane, o, inf, hsc);
+                                else sp_dequant<AFMT, GATEUP, 3>(cur, h, ss, tbl_lane, o, inf, hsc);
+                            } else if constexpr (SS == 2) {
+                                if (J == 0) sp_dequant<AFMT, GATEUP, 0>(cur, h, ss, tbl_lane, o, inf);
+                                else sp_dequant<AFMT, GATEUP, 1>(cur, h, ss, tbl_lane, o, inf);
+                            } else {
+                                sp_dequant<AFMT, GATEUP, 0>(cur, h, ss, tbl_lane, o, inf);
+                            }
+                            st_a(s, m, h, js, o);
                         }
-                        put_a(s, m, h, o);
+                        end_a(s);
                     }
                 }
             }
