@@ -350,9 +350,9 @@ class DeviceLayer:
         out = expert_ffn_decode(self.ex, x, ids, w, self.ws, out=out)
         return (out, ids, w) if return_routing else out
 
-    def decode_graph(self) -> "DecodeGraph":
+    def decode_graph(self, host_io: bool = False) -> "DecodeGraph":
         """A CUDA-graph replay of this layer's single-token decode (route + experts); see DecodeGraph."""
-        return DecodeGraph(self)
+        return DecodeGraph(self, host_io=host_io)
 
     def forward_grouped(self, x: torch.Tensor):
         """Prefill entry: grouped experts then combine (returns out, ids, weights, y_perm, inv_perm)."""
@@ -384,9 +384,15 @@ class DecodeGraph:
     ``x`` (bf16 [1, d]) and ``out`` (fp32 [1, d]) are buffers owned by this object: write the token into ``x``
     (or pass it to ``__call__``), replay, read ``out``.  Replays run on the current stream; consecutive replays
     reuse the same buffers, so read ``out`` before the next one.
+
+    With ``host_io=True`` the graph also holds the two copies: it starts with a copy of the pinned host buffer
+    ``x_host`` (int16 bits of the bf16 token) to the device and ends with a copy of the output to the pinned host
+    buffer ``out_host``, so a decode step from host memory to host memory is one graph launch.  ``__call__``
+    then writes its argument into ``x_host`` (a host copy) and returns ``out_host``, which holds the result once
+    the stream has been synchronized; write the next token only after that synchronization.
     """
 
-    def __init__(self, layer: DeviceLayer):
+    def __init__(self, layer: DeviceLayer, host_io: bool = False):
         s = layer.shape
         dev = layer.device
         self.layer = layer
@@ -398,6 +404,10 @@ class DecodeGraph:
         self.ws = torch.empty(max(workspace_size(layer.ex, 1, s.k), 1), dtype=torch.uint8, device=dev)
         self.route_ws = torch.empty(max(int(lib().ds4moe_route_workspace_size(1, s.d, s.E)), 1), dtype=torch.uint8,
                                     device=dev)
+        self.host_io = host_io
+        if host_io:
+            self.x_host = torch.zeros((1, s.d), dtype=torch.int16).pin_memory()
+            self.out_host = torch.zeros((1, s.d), dtype=torch.float32).pin_memory()
         side = torch.cuda.Stream(device=dev)
         side.wait_stream(torch.cuda.current_stream(dev))
         with torch.cuda.stream(side):
@@ -410,12 +420,21 @@ class DecodeGraph:
 
     def _record(self):
         L = self.layer
+        if self.host_io:
+            self.x.view(torch.int16).copy_(self.x_host, non_blocking=True)
         route(self.x, L.wr, L.bias, L.shape.k, ws=self.route_ws, ids=self.ids, weights=self.weights)
         expert_ffn_decode(L.ex, self.x, self.ids, self.weights, self.ws, out=self.out)
+        if self.host_io:
+            self.out_host.copy_(self.out, non_blocking=True)
 
     def __call__(self, x: Optional[torch.Tensor] = None) -> torch.Tensor:
         """Copy x (bf16 or int16 bits, [1, d], device or pinned host) into the input buffer if given, replay,
         and return the output buffer."""
+        if self.host_io:
+            if x is not None:
+                self.x_host.copy_(x.view(torch.int16))
+            self.graph.replay()
+            return self.out_host
         if x is not None:
             self.x.view(torch.int16).copy_(x.view(torch.int16), non_blocking=True)
         self.graph.replay()

@@ -252,3 +252,20 @@ def test_decode_graph_matches_eager(ds4):
         torch.cuda.synchronize()
         assert ds4.last_device_error() == 0
         assert torch.equal(got, want), t
+
+
+def test_decode_graph_with_host_buffers(ds4):
+    """The graph that also holds the H2D copy of x and the D2H copy of the output gives the same bits as the
+    eager decode, read from its pinned host output buffer after a synchronization."""
+    wl = synth.WORKLOADS["tiny"]
+    L = synth.make_layer(wl)
+    D = ds4.DeviceLayer(L, max_tokens=1)
+    xh = torch.from_numpy(synth.activations(wl, 4, stream=12)).pin_memory()
+    G = D.decode_graph(host_io=True)
+    assert G.out_host.device.type == "cpu" and G.out_host.is_pinned()
+    for t in range(4):
+        want = D.forward(xh[t:t + 1].cuda().view(torch.bfloat16)).cpu()
+        got = G(xh[t:t + 1])
+        torch.cuda.synchronize()
+        assert ds4.last_device_error() == 0
+        assert torch.equal(got, want), t
