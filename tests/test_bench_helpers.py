@@ -44,3 +44,22 @@ def test_step_bytes_counts_each_touched_expert_once():
     assert bench.step_bytes(s, 24, 5) - bench.step_bytes(s, 24, 4) == 4096 * (2 + 4)
     # the B = 1 decode workload touches k experts: the same bytes as the main line's per-token figure
     assert bench.step_bytes(s, s.k, 1) == bench.layer_bytes(synth.WORKLOADS["decode"])
+
+
+def test_every_other_workload_gets_its_own_oracle_baseline(monkeypatch):
+    """workload_cpu_baselines times the oracle on each workload's own layer with a bounded per-thread sample and
+    reports it in the contract's cpu_baseline form (value, unit, cores, kind, sample)."""
+    calls = []
+
+    def fake(wl, n_tokens, nthreads, seed_stream=7):
+        calls.append((wl.name, n_tokens, nthreads))
+        return 10.0 * n_tokens, 0.1
+
+    monkeypatch.setattr(bench, "oracle_tokens_per_s", fake)
+    res = bench.workload_cpu_baselines(4)
+    assert set(res) == {"tiny", "batched", "prefill", "q4"}
+    for name, cb in res.items():
+        assert cb["kind"] == "oracle" and cb["cores"] == 4 and cb["unit"] == bench.UNIT
+        assert cb["value"] > 0 and name in cb["sample"]
+    assert [c[0] for c in calls] == ["tiny", "batched", "prefill", "q4"]
+    assert all(nthreads == 4 and n % 4 == 0 for _, n, nthreads in calls)
