@@ -17,8 +17,9 @@
 //    entry (128-bit lookups without bank conflicts, addressed with one byte
 //    permute); signs XORed onto the fp16 sign bits; packed fp16 FMAs inside a
 //    32-weight group (one scale), fp32 across groups; the row's first lane
-//    writes h_j = silu(g) * u.  Shared-expert row pairs are units as well and
-//    run before the grid-dependency wait (they need neither ids nor the router).
+//    writes h_j = silu(g) * u.  Shared-expert row pairs are units as well (one
+//    row pair each for IQ2X, so the bf16 rows spread over all warps) and run
+//    before the grid-dependency wait (they need neither ids nor the router).
 //  * down (Q2K): byte -> 4 x fp16 table (32 lane slots); h_j staged per expert
 //    as fp16 scaled by a power of two, with sums of every 8 staged values for
 //    the min term; a unit is 2 output rows over all k experts and the shared
@@ -282,7 +283,7 @@ __device__ __forceinline__ float bf16x8_dot(const uint4 w, const float4 a, const
     return s;
 }
 
-// Units of NR row pairs: shared-expert units first (rows NR u .. NR u + NR - 1 of Gs, Us), then routed units
+// Units: shared-expert units first (NRS row pairs of Gs, Us each, see below), then routed units of NR row pairs
 // (expert slot j, rows NR i ..).  Row-matrix index rr = 2 * (row - first row) + (0 gate, 1 up).
 template <int FMT, int VPP, int NR>
 __global__ void __launch_bounds__(DG_THREADS, 1)
@@ -304,14 +305,18 @@ __global__ void __launch_bounds__(DG_THREADS, 1)
 
     constexpr int NRR = 2 * NR;      // row-matrices per unit
     constexpr int LPV = 32 / NRR;    // lanes that hold one row-matrix sum after the reduce-scatter
-    const int n_sh = fs / NR;
+    // Shared-expert units: one row pair for IQ2X rows of d >= 2048 (VPP = 8: d / 256 passes, a multiple of 4),
+    // which spreads the bf16 rows over all warps; Q4K and shorter rows keep NR row pairs (one pass per ring turn).
+    // Either way every pass and ring slot below is in range without run-time guards.
+    constexpr int NRS = FMT == DS4MOE_FMT_Q4K || VPP < 8 ? NR : 1;
+    const int n_sh = fs / NRS;
     const int upe = f / NR;  // routed units per expert
     const int n_all = n_sh + k * upe;
     const int nW = gridDim.x * DG_WARPS;
     const int u_first = warp * gridDim.x + blockIdx.x;
     // the shared expert's rows of this warp's first unit go to L2 while the tables are built
-    if (u_first < n_sh && lane < NRR)
-        prefetch_l2((lane & 1 ? ex.sh_up : ex.sh_gate) + size_t(u_first * NR + (lane >> 1)) * d, uint32_t(d * 2));
+    if (u_first < n_sh && lane < 2 * NRS)
+        prefetch_l2((lane & 1 ? ex.sh_up : ex.sh_gate) + size_t(u_first * NRS + (lane >> 1)) * d, uint32_t(d * 2));
 
     // prologue, one global round trip: every thread loads its codebook entry and its 8 activations together,
     // then writes the codebook table (entry e, lane slot s at DG_TABLE_ABS + e * 256 + s * 16: 8 grid values as
@@ -397,29 +402,38 @@ __global__ void __launch_bounds__(DG_THREADS, 1)
 #pragma unroll
         for (int i = 0; i < NRR; i++) acc[i] = 0.f;
         if (u < n_sh) {
-            // shared expert (bf16): pass p covers elements [256 p, 256 p + 256), lane slice 8 elements; ring of 8 rows
-            const size_t r0 = size_t(u) * NR;
-            const int ns = d / 256, T = ns * NRR;
+            // shared expert (bf16), NRS row pairs: pass p covers elements [256 p, 256 p + 256), lane slice 8
+            // elements; a ring of the next 8 row slices t = p * NRRS + rr (slot t % 8)
+            constexpr int NRRS = 2 * NRS, PU = 8 / NRRS, LPVS = 32 / NRRS;
+            const size_t r0 = size_t(u) * NRS;
+            const int ns = d / 256, T = ns * NRRS;
             auto wptr = [&](int t) {
-                const int rr = t % NRR;
-                return (rr & 1 ? ex.sh_up : ex.sh_gate) + (r0 + (rr >> 1)) * d + (t / NRR) * 256 + lane * 8;
+                const int rr = t % NRRS;
+                return (rr & 1 ? ex.sh_up : ex.sh_gate) + (r0 + (rr >> 1)) * d + (t / NRRS) * 256 + lane * 8;
             };
+            float sacc[NRRS];
+#pragma unroll
+            for (int i = 0; i < NRRS; i++) sacc[i] = 0.f;
             uint4 ring[8];
 #pragma unroll
             for (int s = 0; s < 8; s++) ring[s] = ldg_nc_v4(wptr(s));
-            for (int p = 0; p < ns; p++) {
-                const float4 xa = reinterpret_cast<const float4 *>(x32)[swz16(p * 64 + 2 * lane)];
-                const float4 xb = reinterpret_cast<const float4 *>(x32)[swz16(p * 64 + 2 * lane + 1)];
+            for (int p0 = 0; p0 < ns; p0 += PU) {
 #pragma unroll
-                for (int rr = 0; rr < NRR; rr++) {
-                    acc[rr] += bf16x8_dot(ring[rr & 7], xa, xb);
-                    const int tn = p * NRR + rr + 8;
-                    if (tn < T) ring[rr & 7] = ldg_nc_v4(wptr(tn));
+                for (int q = 0; q < PU; q++) {
+                    const int p = p0 + q;
+                    const float4 xa = reinterpret_cast<const float4 *>(x32)[swz16(p * 64 + 2 * lane)];
+                    const float4 xb = reinterpret_cast<const float4 *>(x32)[swz16(p * 64 + 2 * lane + 1)];
+#pragma unroll
+                    for (int rr = 0; rr < NRRS; rr++) {
+                        sacc[rr] += bf16x8_dot(ring[q * NRRS + rr], xa, xb);
+                        const int tn = p * NRRS + rr + 8;
+                        if (tn < T) ring[q * NRRS + rr] = ldg_nc_v4(wptr(tn));
+                    }
                 }
             }
-            const float v = reduce_scatter<NRR>(acc, lane);
-            const float up = __shfl_xor_sync(0xffffffffu, v, LPV);  // gate of row i on lane 2 i LPV, up next
-            if (lane % (2 * LPV) == 0) hs_out[r0 + lane / (2 * LPV)] = silu(v) * up;
+            const float v = reduce_scatter<NRRS>(sacc, lane);
+            const float up = __shfl_xor_sync(0xffffffffu, v, LPVS);  // gate of row i on lane 2 i LPVS, up next
+            if (lane % (2 * LPVS) == 0) hs_out[r0 + lane / (2 * LPVS)] = silu(v) * up;
             continue;
         }
         if (!waited) {
@@ -484,12 +498,16 @@ constexpr uint32_t DD_TABLE_ABS = 0x10000;  // absolute shared address of the 64
 constexpr int DD_ROWS = 2;                  // output rows per unit
 
 // Contraction lengths (f) the down kernel takes: f = 256 * 2^i up to 8192.  A lane owns EPL = min(64, f / 32)
-// consecutive weights of a row per pass; f / (32 EPL) passes.
+// consecutive weights of a row per pass for Q2K, min(32, f / 32) for Q4K (whose 64-weight slices, 32 bytes of
+// codes plus 16 of scales per row, spill at 128 registers); f / (32 EPL) passes.
 __host__ __device__ __forceinline__ bool dd_supported_f(int f) {
     const int nblk = f / QK;
     return f % QK == 0 && nblk >= 1 && nblk <= 32 && (nblk & (nblk - 1)) == 0;
 }
-__host__ __device__ __forceinline__ int dd_epl(int f) { return f / 32 < 64 ? f / 32 : 64; }
+__host__ __device__ __forceinline__ int dd_epl(int f, int fmt) {
+    const int cap = fmt == DS4MOE_FMT_Q4K ? 32 : 64;
+    return f / 32 < cap ? f / 32 : cap;
+}
 
 // Staged h is stored per lane slice (the EPL weights one lane owns in one pass), each slice padded by 16 bytes
 // when that keeps the 8 lanes of a quarter-warp on distinct banks; the lane then reads its slice with
@@ -497,9 +515,9 @@ __host__ __device__ __forceinline__ int dd_epl(int f) { return f / 32 < 64 ? f /
 struct DownSmemLayout {
     int hq, hq_sb, hq_eb, hsum, hs_sb, hs_eb, hs, wsc, eid, total;  // byte offsets from the table base / strides
 };
-__host__ __device__ __forceinline__ DownSmemLayout dd_layout(int k, int f, int fs) {
+__host__ __device__ __forceinline__ DownSmemLayout dd_layout(int k, int f, int fs, int fmt) {
     DownSmemLayout L;
-    const int epl = dd_epl(f);
+    const int epl = dd_epl(f, fmt);
     const int nsl = f / epl;                           // lane slices per expert (32 per pass)
     L.hq_sb = epl * 2 + (epl >= 16 ? 16 : 0);
     L.hq_eb = nsl * L.hq_sb;
@@ -683,7 +701,7 @@ __global__ void __launch_bounds__(DD_THREADS, 1)
     const int npass = f / (32 * EPL);
     const uint32_t sbase = smem_u32(smem);
     uint8_t *tb = smem + (DD_TABLE_ABS - sbase);
-    const DownSmemLayout L = dd_layout(k, f, fs);
+    const DownSmemLayout L = dd_layout(k, f, fs, FMT);
     float *hsl = reinterpret_cast<float *>(tb + L.hs);
     float *wsc = reinterpret_cast<float *>(tb + L.wsc);
     int *eid = reinterpret_cast<int *>(tb + L.eid);
@@ -748,11 +766,61 @@ __global__ void __launch_bounds__(DD_THREADS, 1)
             }
     };
 
-    // stage h_j (one warp per expert): fp16 of h * 2^e_j with max |h_j| * 2^e_j in [32, 64), and the fp32 sums of
-    // every 8 staged values, both in per-lane-slice order.  Loads go out 4 per lane at a time.
-    for (int j = warp; j < k; j += DD_WARPS) {
+    // Stage h_j: fp16 of h * 2^e_j with max |h_j| * 2^e_j in [32, 64), and the fp32 sums of every 8 staged values,
+    // both in per-lane-slice order.  With k <= 8 experts and f <= 2048 two warps share an expert and hold their
+    // halves in registers (one round of loads, all 16 warps busy); otherwise one warp per expert loads its chunks
+    // twice (for the maximum, then to convert), 4 per lane at a time.  The result is the same either way.
+    const int nc = f / 128;  // float4 chunks of h_j per lane (a multiple of 2)
+    // h_j -> fp16 slice of one chunk c (weights 4c .. 4c + 3 of lane slice order), and its sums of 8
+    auto stage_chunk = [&](int j, int c, float4 v, float sc) {
+        const __half2 p0 = __floats2half2_rn(v.x * sc, v.y * sc);
+        const __half2 p1 = __floats2half2_rn(v.z * sc, v.w * sc);
+        const int el = 4 * c, slice = el / EPL, o = el % EPL;  // slice = pass * 32 + lane
+        *reinterpret_cast<uint2 *>(tb + L.hq + j * L.hq_eb + slice * L.hq_sb + o * 2) =
+            make_uint2(half2_as_u32(p0), half2_as_u32(p1));
+        const float2 a = __half22float2(p0), b = __half22float2(p1);
+        float s = (a.x + a.y) + (b.x + b.y);
+        s += __shfl_xor_sync(0xffffffffu, s, 1);
+        if ((lane & 1) == 0)
+            *reinterpret_cast<float *>(tb + L.hsum + j * L.hs_eb + slice * L.hs_sb + (o / 8) * 4) = s;
+    };
+    auto expert_meta = [&](int j, int e) {
+        wsc[j] = wts[j] * ldexpf(1.f, -e);
+        const int id = ids[j];
+        eid[j] = id;
+        if (id < 0 || id >= ex.E) set_device_error(DS4MOE_EDEVICE);
+    };
+    const bool two_warps = 2 * k <= DD_WARPS && nc <= 16;  // uniform over the block
+    if (two_warps) {
+        // two warps per expert, each holding its half of h_j's chunks in registers (one round of loads); the
+        // halves' maxima meet in shared memory
+        __shared__ float s_hmax[DD_WARPS];
+        const int j = warp >> 1, hf = warp & 1, nh = nc / 2;
+        float4 v[8];
+        if (j < k) {
+            const float4 *hj = reinterpret_cast<const float4 *>(h + size_t(j) * f) + hf * nh * 32;
+#pragma unroll
+            for (int i = 0; i < 8; i++)
+                if (i < nh) v[i] = hj[i * 32 + lane];
+            float m = 0.f;
+#pragma unroll
+            for (int i = 0; i < 8; i++)
+                if (i < nh) m = fmaxf(m, fmaxf(fmaxf(fabsf(v[i].x), fabsf(v[i].y)), fmaxf(fabsf(v[i].z), fabsf(v[i].w))));
+            m = warp_max(m);
+            if (lane == 0) s_hmax[warp] = m;
+        }
+        __syncthreads();
+        if (j < k) {
+            const int e = pow2_exponent_for(fmaxf(s_hmax[2 * j], s_hmax[2 * j + 1]), 6);
+            const float sc = ldexpf(1.f, e);
+#pragma unroll
+            for (int i = 0; i < 8; i++)
+                if (i < nh) stage_chunk(j, (hf * nh + i) * 32 + lane, v[i], sc);
+            if (hf == 0 && lane == 0) expert_meta(j, e);
+        }
+    }
+    for (int j = warp; j < k && !two_warps; j += DD_WARPS) {
         const float4 *hj = reinterpret_cast<const float4 *>(h + size_t(j) * f);
-        const int nc = f / 128;  // float4 chunks per lane (a multiple of 2)
         float m = 0.f;
         for (int c0 = 0; c0 < nc; c0 += 4) {
             float4 v[4];
@@ -772,28 +840,10 @@ __global__ void __launch_bounds__(DD_THREADS, 1)
             for (int i = 0; i < 4; i++)
                 if (c0 + i < nc) v[i] = hj[(c0 + i) * 32 + lane];
 #pragma unroll
-            for (int i = 0; i < 4; i++) {
-                if (c0 + i < nc) {
-                    const int c = (c0 + i) * 32 + lane;  // weights 4c .. 4c+3
-                    const __half2 p0 = __floats2half2_rn(v[i].x * sc, v[i].y * sc);
-                    const __half2 p1 = __floats2half2_rn(v[i].z * sc, v[i].w * sc);
-                    const int el = 4 * c, slice = el / EPL, o = el % EPL;  // slice = pass * 32 + lane
-                    *reinterpret_cast<uint2 *>(tb + L.hq + j * L.hq_eb + slice * L.hq_sb + o * 2) =
-                        make_uint2(half2_as_u32(p0), half2_as_u32(p1));
-                    const float2 a = __half22float2(p0), b = __half22float2(p1);
-                    float s = (a.x + a.y) + (b.x + b.y);
-                    s += __shfl_xor_sync(0xffffffffu, s, 1);
-                    if ((lane & 1) == 0)
-                        *reinterpret_cast<float *>(tb + L.hsum + j * L.hs_eb + slice * L.hs_sb + (o / 8) * 4) = s;
-                }
-            }
+            for (int i = 0; i < 4; i++)
+                if (c0 + i < nc) stage_chunk(j, (c0 + i) * 32 + lane, v[i], sc);
         }
-        if (lane == 0) {
-            wsc[j] = wts[j] * ldexpf(1.f, -e);
-            const int id = ids[j];
-            eid[j] = id;
-            if (id < 0 || id >= ex.E) set_device_error(DS4MOE_EDEVICE);
-        }
+        if (lane == 0) expert_meta(j, e);
     }
     for (int i = tid * 4; i < fs; i += DD_THREADS * 4)
         reinterpret_cast<float4 *>(hsl)[swz16(i / 4)] = *reinterpret_cast<const float4 *>(hs_in + i);

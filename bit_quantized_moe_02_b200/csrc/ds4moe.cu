@@ -188,7 +188,7 @@ bool decode_gemv_supported(const ds4moe_experts *ex, int k) {
     const bool q4 = ex->fmt_gate == DS4MOE_FMT_Q4K && ex->fmt_down == DS4MOE_FMT_Q4K;
     if (!(iq || q4) || k > 32) return false;
     if (!dg_supported_d(ex->d) || !dd_supported_f(ex->f)) return false;
-    return dd_layout(k, ex->f, ex->f_shared).total <= 200 * 1024;
+    return dd_layout(k, ex->f, ex->f_shared, ex->fmt_down).total <= 200 * 1024;
 }
 
 // Decode batches of up to this many tokens run the single-token GEMV pair once per token (each pass streams its
@@ -657,13 +657,13 @@ ds4moe_status ds4moe_decode_down(const ds4moe_experts *ex, const int32_t *ids, c
     const ExpertsDev D = to_dev(ex);
     const float *h = reinterpret_cast<const float *>(w8 + W.h);
     const float *hs = reinterpret_cast<const float *>(w8 + W.hs);
-    const int smem = dd_layout(k, ex->f, ex->f_shared).total;
-    const int epl = dd_epl(ex->f);  // weights of a row per lane and pass
+    const int smem = dd_layout(k, ex->f, ex->f_shared, ex->fmt_down).total;
+    const int epl = dd_epl(ex->f, ex->fmt_down);  // weights of a row per lane and pass
     using DK = void (*)(const ExpertsDev, const float *, const float *, const int32_t *, const float *, int, float *);
     DK kern;
     if (ex->fmt_down == DS4MOE_FMT_Q4K)
-        kern = epl == 64 ? decode_down_kernel<DS4MOE_FMT_Q4K, 64> : epl == 32 ? decode_down_kernel<DS4MOE_FMT_Q4K, 32>
-             : epl == 16 ? decode_down_kernel<DS4MOE_FMT_Q4K, 16> : decode_down_kernel<DS4MOE_FMT_Q4K, 8>;
+        kern = epl == 32 ? decode_down_kernel<DS4MOE_FMT_Q4K, 32> : epl == 16 ? decode_down_kernel<DS4MOE_FMT_Q4K, 16>
+                         : decode_down_kernel<DS4MOE_FMT_Q4K, 8>;
     else
         kern = epl == 64 ? decode_down_kernel<DS4MOE_FMT_Q2K, 64> : epl == 32 ? decode_down_kernel<DS4MOE_FMT_Q2K, 32>
              : epl == 16 ? decode_down_kernel<DS4MOE_FMT_Q2K, 16> : decode_down_kernel<DS4MOE_FMT_Q2K, 8>;
