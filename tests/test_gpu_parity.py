@@ -183,6 +183,18 @@ def test_decode_gemv_shapes(ds4, d, f, fs, E, k):
     run_and_compare(ds4, L, x, "decode")
 
 
+@pytest.mark.parametrize("d,f,fs,E,k,fmt", [(1024, 4096, 512, 16, 4, "iq2x"), (1024, 512, 256, 32, 12, "iq2x"),
+                                              (1024, 4096, 512, 16, 4, "q4k")])
+def test_decode_gemv_one_warp_staging(ds4, d, f, fs, E, k, fmt):
+    """Single-token decode where the down kernel stages each expert's h with one warp (f > 2048, or k > 8 experts,
+    so two warps per expert do not fit): the other staging path of the GEMV down kernel."""
+    f3 = {"fmt_gate": "q4k", "fmt_up": "q4k", "fmt_down": "q4k"} if fmt == "q4k" else {}
+    shape = synth.LayerShape(d=d, E=E, f=f, k=k, f_shared=fs, **f3)
+    L = layer_of(shape, 1.0, 51 + f + k)
+    x = synth.f32_to_bf16_bits(synth.rng(9, d, f, k).normal(size=(2, d)).astype(np.float32))
+    run_and_compare(ds4, L, x, "decode")
+
+
 @pytest.mark.parametrize("d,f,fs,E,k", [(4096, 2048, 2048, 16, 8), (2048, 1024, 512, 16, 4), (1024, 256, 0, 8, 2)])
 def test_q4k_decode_gemv(ds4, d, f, fs, E, k):
     """Single-token decode of Q4K layers through the GEMV kernels (the decode layer's shape with 16 experts, then
